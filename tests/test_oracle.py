@@ -1,0 +1,309 @@
+"""Pins of the fp64 oracle against facts outside itself (CPU only).
+
+Each test names what it pins: a value the pages print, an identity the pages
+state, a library routine (torch SDPA in fp64), a closed form, or brute force.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from depth_planed_kv_b200 import synth as S
+from oracle import oracle as OR
+from tests.util import all_depth_rows, branch_rows, seq_planes
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def small(R=4, H=2, d=16, W=8, k=4, decay=0.88, seed=7, dtype="f32"):
+    return S.Workload("t", 1, R, H, d, W, k, 1, None, decay, seed, dtype, 256, k)
+
+
+def run_oracle(wl, T, ws, k, mode=1, layer=0, seq=3, nseq=1):
+    seqs = [seq_planes(wl, layer, seq + s, T, ws) for s in range(nseq)]
+    table, Q, Kb, Vb = all_depth_rows(wl, layer, nseq, [seq + s for s in range(nseq)], k)
+    O, lse = OR.verify(seqs, table, Q, Kb, Vb, 1 / math.sqrt(wl.d), mode)
+    return O, lse, (seqs, table, Q, Kb, Vb)
+
+
+def sdpa_row(q, keys, vals, scale):
+    """torch SDPA in fp64 on an explicitly gathered key list (library routine)."""
+    qt = torch.from_numpy(np.asarray(q, np.float64)).view(1, 1, 1, -1)
+    kt = torch.from_numpy(np.asarray(keys, np.float64)).view(1, 1, len(keys), -1)
+    vt = torch.from_numpy(np.asarray(vals, np.float64)).view(1, 1, len(vals), -1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+    return o.view(-1).numpy()
+
+
+def full_planes(wl, layer, seq, T):
+    """Every plane 1..R of every position 0..T-1: [H][R][T][d] (the full cache)."""
+    coef = S.coef_table(wl.decay, wl.R)
+    k = S.planes(wl.seed, 0, layer, seq, range(wl.H), np.arange(1, wl.R + 1), np.arange(T), wl.d,
+                 wl.R, coef, wl.bf16)
+    v = S.planes(wl.seed, 1, layer, seq, range(wl.H), np.arange(1, wl.R + 1), np.arange(T), wl.d,
+                 wl.R, coef, wl.bf16)
+    return k, v
+
+
+# --- P1: the page's memory figure --------------------------------------------------
+
+def test_memory_fraction_matches_printed_value():
+    g = json.load(open(os.path.join(GOLDEN, "memory_fraction.json")))
+    f = OR.memory_fraction(g["T"], g["W"], g["R"], g["n_recurrent"], g["n_prelude"], g["n_coda"])
+    assert round(100 * f, g["printed_decimals"]) == g["printed_percent"]
+
+
+def test_memory_fraction_limits_and_store_count():
+    # W >= T keeps everything; the store model's live-plane count equals the model.
+    assert OR.memory_fraction(1024, 1024, 32, 4, 2, 2) == 1.0
+    assert OR.memory_fraction(1024, 4096, 32, 4, 2, 2) == 1.0
+    # W = 0 keeps one plane per position per layer
+    assert OR.memory_fraction(1024, 0, 32, 4, 2, 2) == pytest.approx(8 / (4 + 4 * 32))
+    for W in (0, 4, 64, 256, 1024):
+        st = OR.OracleStore(1, 32, 1, 8, W, 1024 + 8, 1, 8, np.float32)
+        K = np.zeros((1, 1, 1024, 32, 1, 8), np.float32)
+        st.append([0], [1024], K, K)
+        st.evict([0])
+        live = st.live_planes(0)
+        assert live / (32 * 1024) == pytest.approx(OR.memory_fraction(1024, W, 32, 1))
+
+
+# --- P5: brute force, the library routine, closed forms ----------------------------
+
+def test_naive_and_region_agree():
+    wl = small()
+    for T, ws in [(48, 40), (48, 0), (48, 48), (48, 60), (0, 0), (5, 2), (1, 1)]:
+        O0, l0, _ = run_oracle(wl, T, ws, 4, mode=0, nseq=2)
+        O1, l1, _ = run_oracle(wl, T, ws, 4, mode=1, nseq=2)
+        assert np.abs(O0 - O1).max() < 1e-13
+        assert np.abs(l0 - l1).max() < 1e-12
+
+
+def test_against_torch_sdpa_on_gathered_keys():
+    wl = small(R=5, H=3, d=8)
+    T, ws, k = 20, 13, 3
+    O, lse, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, ws, k)
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            for h in range(wl.H):
+                keys = [kf[h, (r if p >= ws else wl.R) - 1, p] for p in range(T)]
+                vals = [vf[h, (r if p >= ws else wl.R) - 1, p] for p in range(T)]
+                keys += [Kb[row0 + jj * stride, h] for jj in range(j + 1)]
+                vals += [Vb[row0 + jj * stride, h] for jj in range(j + 1)]
+                ref = sdpa_row(Q[row, h], keys, vals, scale)
+                assert np.abs(O[row, h] - ref).max() < 1e-13
+
+
+def test_pure_python_brute_force():
+    wl = small(R=3, H=1, d=4, W=2, k=2, seed=11)
+    T, ws, k = 5, 3, 2
+    O, lse, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, ws, k)
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            q = [float(x) for x in Q[row, 0]]
+            keys, vals = [], []
+            for p in range(T):
+                plane = r if p >= ws else wl.R
+                keys.append([float(x) for x in kf[0, plane - 1, p]])
+                vals.append([float(x) for x in vf[0, plane - 1, p]])
+            for jj in range(j + 1):
+                keys.append([float(x) for x in Kb[row0 + jj * stride, 0]])
+                vals.append([float(x) for x in Vb[row0 + jj * stride, 0]])
+            s = [scale * sum(a * b for a, b in zip(q, kk)) for kk in keys]
+            e = [math.exp(x) for x in s]
+            z = sum(e)
+            o = [sum(e[t] * vals[t][c] for t in range(len(e))) / z for c in range(wl.d)]
+            assert max(abs(O[row, 0, c] - o[c]) for c in range(wl.d)) < 1e-12
+            assert abs(lse[row, 0] - math.log(z)) < 1e-12
+
+
+def test_closed_forms():
+    wl = small()
+    T, ws, k = 30, 26, 4
+    O, lse, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, ws, k)
+    scale = 1 / math.sqrt(wl.d)
+    # single key: empty prefix, first token sees only itself -> o = v, lse = s
+    O1, l1 = OR.verify([dict(seqs[0], T=0, ws=0, Kd=seqs[0]["Kd"][:, :0], Vd=seqs[0]["Vd"][:, :0],
+                             Kw=seqs[0]["Kw"][:, :, :0], Vw=seqs[0]["Vw"][:, :, :0])],
+                       table, Q, Kb, Vb, scale)
+    for (seq, r, n, row0, stride) in table:
+        assert np.array_equal(O1[row0], Vb[row0].astype(np.float64))
+        np.testing.assert_allclose(l1[row0], scale * np.sum(Q[row0].astype(np.float64)
+                                                            * Kb[row0], axis=-1), rtol=0, atol=1e-14)
+    # equal scores (q = 0): o = mean of the visible values, lse = ln(#keys)
+    Oz, lz = OR.verify(seqs, table, np.zeros_like(Q), Kb, Vb, scale)
+    kd_v = seqs[0]["Vd"].astype(np.float64)
+    kw_v = seqs[0]["Vw"].astype(np.float64)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            vis = [kd_v[:, p] if (p < ws or r == wl.R) else kw_v[:, r - 1, p - ws] for p in range(T)]
+            vis += [Vb[row0 + jj * stride].astype(np.float64) for jj in range(j + 1)]
+            np.testing.assert_allclose(Oz[row], np.mean(vis, axis=0), rtol=0, atol=1e-14)
+            np.testing.assert_allclose(lz[row], math.log(T + j + 1), rtol=0, atol=1e-14)
+    # V == 1 everywhere: every output is exactly 1 up to rounding (rows sum to 1)
+    ones = lambda a: np.ones_like(a)
+    s1 = [dict(seqs[0], Vd=ones(seqs[0]["Vd"]), Vw=ones(seqs[0]["Vw"]))]
+    O_1, _ = OR.verify(s1, table, Q, Kb, ones(Vb), scale)
+    assert np.abs(O_1 - 1).max() < 1e-14
+
+
+# --- P2 / P3: the window identities --------------------------------------------------
+
+@pytest.mark.parametrize("R", [1, 4])
+def test_window_covering_context_is_full_cache(R):
+    wl = small(R=R, H=2, d=8)
+    T, k = 24, 3
+    O, _, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, 0, k)  # ws = 0: all positions in window
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            for h in range(wl.H):
+                keys = list(kf[h, r - 1]) + [Kb[row0 + jj * stride, h] for jj in range(j + 1)]
+                vals = list(vf[h, r - 1]) + [Vb[row0 + jj * stride, h] for jj in range(j + 1)]
+                assert np.abs(O[row, h] - sdpa_row(Q[row, h], keys, vals, scale)).max() <= 1e-13
+
+
+def test_zero_window_is_deepest_plane_only():
+    wl = small(R=4, H=2, d=8)
+    T, k = 24, 3
+    O, _, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, T, k)  # ws = T: nothing in window
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            for h in range(wl.H):
+                keys = list(kf[h, wl.R - 1]) + [Kb[row0 + jj * stride, h] for jj in range(j + 1)]
+                vals = list(vf[h, wl.R - 1]) + [Vb[row0 + jj * stride, h] for jj in range(j + 1)]
+                assert np.abs(O[row, h] - sdpa_row(Q[row, h], keys, vals, scale)).max() <= 1e-13
+
+
+def test_single_plane_is_ordinary_causal_attention():
+    wl = small(R=1, H=2, d=8)
+    T, k = 17, 4
+    O, _, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, 9, k)
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    q = torch.from_numpy(Q.astype(np.float64)).permute(1, 0, 2)[None]            # [1,H,k,d]
+    kk = torch.from_numpy(np.concatenate([kf[:, 0], np.transpose(Kb, (1, 0, 2))], 1).astype(np.float64))[None]
+    vv = torch.from_numpy(np.concatenate([vf[:, 0], np.transpose(Vb, (1, 0, 2))], 1).astype(np.float64))[None]
+    mask = torch.ones(k, T + k, dtype=torch.bool).tril(diagonal=T)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, kk, vv, attn_mask=mask, scale=scale)
+    assert np.abs(O - ref[0].permute(1, 0, 2).numpy()).max() <= 1e-13
+
+
+# --- P6: block independence ---------------------------------------------------------
+
+def test_rows_ignore_other_depths_and_later_tokens():
+    wl = small(R=4, H=2, d=8)
+    T, ws, k = 20, 12, 4
+    O, lse, (seqs, table, Q, Kb, Vb) = run_oracle(wl, T, ws, k)
+    R = wl.R
+    j0, r0 = 1, 2
+    Kp, Vp = Kb.copy(), Vb.copy()
+    rng = np.random.default_rng(0)
+    for j in range(k):
+        for r in range(1, R + 1):
+            if r != r0 or j > j0:
+                row = j * R + (r - 1)
+                Kp[row] += rng.standard_normal(Kp[row].shape).astype(np.float32)
+                Vp[row] += rng.standard_normal(Vp[row].shape).astype(np.float32)
+    O2, l2 = OR.verify(seqs, table, Q, Kp, Vp, 1 / math.sqrt(wl.d))
+    for j in range(j0 + 1):
+        row = j * R + (r0 - 1)
+        assert np.array_equal(O[row], O2[row]) and np.array_equal(lse[row], l2[row])
+    assert not np.array_equal(O, O2)
+
+
+@pytest.mark.parametrize("W", [4, 6, 16])
+def test_batched_equals_one_token_at_a_time(W):
+    """Verifying k tokens in one call == k calls of one token, where tokens 0..j-1
+    were appended with all R planes (no evict) before token j."""
+    wl = small(R=4, H=2, d=8, W=W, k=4)
+    T, k, R = 21, 4, 4
+    seq = 3
+    coef = S.coef_table(wl.decay, R)
+    st = OR.OracleStore(1, R, wl.H, wl.d, W, 64, 8, k, np.float64)
+    allp = np.arange(T)
+    K = np.transpose(S.planes(wl.seed, 0, 0, seq, range(wl.H), np.arange(1, R + 1), allp, wl.d, R,
+                              coef, False), (2, 1, 0, 3))[None, None]     # [1][1][T][R][H][d]
+    V = np.transpose(S.planes(wl.seed, 1, 0, seq, range(wl.H), np.arange(1, R + 1), allp, wl.d, R,
+                              coef, False), (2, 1, 0, 3))[None, None]
+    st.append([seq], [T], K, V)
+    st.evict([seq])
+    scale = 1 / math.sqrt(wl.d)
+    table, Q, Kb, Vb = all_depth_rows(wl, 0, 1, [seq], k)
+    views = [st.plane_view(0, b) for b in range(8)]
+    tb = table.copy()
+    tb[:, 0] = seq
+    Ob, lb = OR.verify(views, tb, Q, Kb, Vb, scale)
+    Kblk = Kb.reshape(k, R, wl.H, wl.d)
+    Vblk = Vb.reshape(k, R, wl.H, wl.d)
+    for j in range(k):
+        s2 = OR.OracleStore(1, R, wl.H, wl.d, W, 64, 8, k, np.float64)
+        s2.append([seq], [T], K, V)
+        s2.evict([seq])
+        if j:
+            s2.append([seq], [j], Kblk[None, None, :j], Vblk[None, None, :j])
+        v2 = [s2.plane_view(0, b) for b in range(8)]
+        for r in range(1, R + 1):
+            row = j * R + (r - 1)
+            one = np.array([[seq, r, 1, 0, 1]], np.int32)
+            O1, l1 = OR.verify(v2, one, Q[row:row + 1], Kb[row:row + 1], Vb[row:row + 1], scale)
+            assert np.abs(O1[0] - Ob[row]).max() <= 1e-13
+            assert np.abs(l1[0] - lb[row]).max() <= 1e-12
+
+
+@pytest.mark.parametrize("W,k", [(4, 4), (8, 4), (3, 4), (1, 8)])
+def test_accepted_block_keeps_all_planes_iff_window_covers_it(W, k):
+    R, H, d = 4, 2, 8
+    st = OR.OracleStore(1, R, H, d, W, 64, 2, k, np.float64)
+    rng = np.random.default_rng(1)
+    K0 = rng.standard_normal((1, 1, 10, R, H, d))
+    st.append([1], [10], K0, K0)
+    st.evict([1])
+    Kb = rng.standard_normal((1, 1, k, R, H, d))
+    Vb = rng.standard_normal((1, 1, k, R, H, d))
+    st.append([1], [k], Kb, Vb)
+    st.evict([1])
+    T, ws = int(st.length[1]), int(st.wstart[1])
+    for t in range(k):
+        p = 10 + t
+        live = p >= ws
+        assert live == (t >= k - W)
+        assert np.array_equal(st.kdeep[0, 1, :, p], Kb[0, 0, t, R - 1])
+        if live:
+            slot = p % st.Wcap
+            assert np.array_equal(st.kwin[0, 1, :, :, slot], np.swapaxes(Kb[0, 0, t, :R - 1], 0, 1))
+            assert np.array_equal(st.vwin[0, 1, :, :, slot], np.swapaxes(Vb[0, 0, t, :R - 1], 0, 1))
+
+
+@pytest.mark.parametrize("W,k", [(4, 4), (64, 4), (8, 8), (3, 4), (1, 4), (7, 8)])
+def test_sliding_reading_block_independent_iff_window_covers_block(W, k):
+    deep = OR.sliding_block_reads_deepest(W, k)
+    assert (not deep.any()) == (W >= k)
+
+
+# --- P7: the generator's planes approach the deepest one as the page says -------
+
+@pytest.mark.parametrize("key", ["huginn_per_loop", "raven_per_loop"])
+def test_generator_decay(key):
+    decay = json.load(open(os.path.join(GOLDEN, "plane_decay.json")))[key]
+    R = 32
+    coef = S.coef_table(decay, R)
+    P = S.planes(5, 0, 0, 0, range(4), np.arange(1, R + 1), np.arange(256), 64, R, coef, False)
+    dist = np.sqrt(((P - P[:, R - 1:R]) ** 2).sum(axis=(0, 2, 3)))
+    ratios = dist[0:R - 2] / dist[1:R - 1]   # distance to plane R shrinks by `decay` per loop
+    assert np.all(np.abs(ratios - decay) < 0.02)
