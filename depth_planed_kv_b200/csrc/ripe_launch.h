@@ -1,0 +1,34 @@
+// ripe_launch.h -- host-side launchers of the libripe kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+struct ripe_cache_s;
+struct BranchArgs;
+
+cudaError_t launch_append(const ripe_cache_s* c, const int32_t* seq_ids, const int32_t* n_acc, int nseq,
+                          const void* K, const void* V, int kmax_in, cudaStream_t st);
+cudaError_t launch_evict(const ripe_cache_s* c, const int32_t* seq_ids, int nseq, cudaStream_t st);
+cudaError_t launch_reset(const ripe_cache_s* c, const int32_t* seq_ids, int nseq, cudaStream_t st);
+cudaError_t launch_truncate(const ripe_cache_s* c, const int32_t* seq_ids, const int32_t* new_len, int nseq,
+                            cudaStream_t st);
+cudaError_t launch_synth_fill(const ripe_cache_s* c, int b, int T, uint64_t seed, const float* coef,
+                              cudaStream_t st);
+
+// Verify plan: how the deep region is split and how much scratch the call needs.
+struct VerifyPlan {
+    int nsplit;        // deep-region splits (partials 0..nsplit-1); the window+block partial is nsplit
+    int chunk;         // keys per deep split
+    int rows_chunk;    // rows per CTA of the window kernel
+    int nrowchunks;    // row chunks per branch
+    int max_ntok;      // host bound on tokens per branch
+    bool tc_deep;      // deep region on the tcgen05 stacked-query kernel
+    size_t work_bytes; // scratch needed
+};
+
+VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths);
+
+cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
+                          const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,
+                          void* O, float* lse, void* work, cudaStream_t st);

@@ -1,0 +1,27 @@
+// ripe_verify.cuh -- argument block shared by the verify kernels.
+#pragma once
+
+#include "ripe_internal.cuh"
+
+struct VerifyArgs {
+    StoreView s;
+    BranchArgs ba;
+    int layer;
+    const char *Q, *Kb, *Vb;  // [nrows][H][d], cache dtype
+    char* O;                  // [nrows][H][d], cache dtype
+    float* lse;               // [nrows][H] or NULL
+    const int32_t* ctx;       // per-sequence context length or NULL
+    float scale_log2;         // softmax scale * log2(e)
+    int nsplit, chunk, nseg;  // deep splits, keys per split, nsplit + 1
+    int nrowchunks;           // row chunks per branch in the CUDA-core kernel
+    float2* part_ml;          // [nrows][H][nseg] (m in log2 units, l)
+    float* part_o;            // [nrows][H][nseg][d]
+};
+
+// Scratch layout: the (m, l) pairs, padded to 256 bytes, then the o vectors.
+inline size_t verify_ml_bytes(int nrows, int H, int nseg) {
+    return ((size_t)nrows * H * nseg * sizeof(float2) + 255) / 256 * 256;
+}
+inline size_t verify_work_bytes(int nrows, int H, int d, int nseg) {
+    return verify_ml_bytes(nrows, H, nseg) + (size_t)nrows * H * nseg * d * sizeof(float);
+}
