@@ -132,6 +132,16 @@ int verify_common(ripe_cache_s* c, int layer, const BranchArgs& ba, const void* 
 
 void ripe_count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+int ripe_fail(int status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
 extern "C" {
 
 const char* ripe_error_string(int status) {

@@ -32,3 +32,6 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
                           const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,
                           void* O, float* lse, void* work, cudaStream_t st);
+
+// Record a one-line message for ripe_last_error() and return `status`.
+int ripe_fail(int status, const char* fmt, ...);

@@ -64,6 +64,8 @@ _sig("ripe_evict", [_P, _P, _I, _P])
 _sig("ripe_truncate", [_P, _P, _P, _I, _P])
 _sig("ripe_verify_attn", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
 _sig("ripe_verify_attn_all_depths", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
+_sig("ripe_verify_attn_noalloc", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P,
+                                  ctypes.POINTER(ctypes.c_size_t)])
 _sig("ripe_reserve_workspace", [_P, _I])
 _sig("ripe_synth_fill", [_P, _P, _P, _I, ctypes.c_uint64, _P, _P])
 _sig("ripe_cache_buffers", [_P] + [ctypes.POINTER(_P)] * 6)
@@ -75,7 +77,8 @@ _sig("ripe_last_error", [], ctypes.c_char_p)
 
 EXPORTED = ["ripe_cache_bytes", "ripe_cache_create", "ripe_cache_destroy", "ripe_cache_reset",
             "ripe_append", "ripe_evict", "ripe_truncate", "ripe_verify_attn",
-            "ripe_verify_attn_all_depths", "ripe_reserve_workspace", "ripe_synth_fill",
+            "ripe_verify_attn_all_depths", "ripe_verify_attn_noalloc", "ripe_reserve_workspace",
+            "ripe_synth_fill",
             "ripe_cache_buffers", "ripe_read_meta", "ripe_get_device_error", "ripe_launch_count",
             "ripe_error_string", "ripe_last_error"]
 
@@ -191,6 +194,20 @@ class RipeCache:
         _check(_lib.ripe_verify_attn(self.handle, layer, _ptr(branches), nbranch, nrows, _ptr(Q),
                                      _ptr(Kblk), _ptr(Vblk), _ptr(ctx_len), ctypes.c_float(scale),
                                      _ptr(O), _ptr(lse), _stream(stream)), "ripe_verify_attn")
+
+    def ripe_verify_attn_noalloc(self, layer: int, branches: torch.Tensor, nbranch: int, Q: torch.Tensor,
+                                 Kblk: torch.Tensor, Vblk: torch.Tensor, O: torch.Tensor,
+                                 lse: Optional[torch.Tensor] = None, ctx_len: Optional[torch.Tensor] = None,
+                                 scale: float = 0.0, stream=None, check: bool = True):
+        """Same as ripe_verify_attn, with the library's fixed scratch instead of an
+        allocation.  Returns (status, scratch bytes used or needed)."""
+        need = ctypes.c_size_t()
+        rc = _lib.ripe_verify_attn_noalloc(self.handle, layer, _ptr(branches), nbranch, Q.shape[0], _ptr(Q),
+                                           _ptr(Kblk), _ptr(Vblk), _ptr(ctx_len), ctypes.c_float(scale),
+                                           _ptr(O), _ptr(lse), _stream(stream), ctypes.byref(need))
+        if check:
+            _check(rc, "ripe_verify_attn_noalloc")
+        return rc, need.value
 
     def ripe_verify_attn_all_depths(self, layer: int, seq_ids: torch.Tensor, k: int, Q: torch.Tensor,
                                     Kblk: torch.Tensor, Vblk: torch.Tensor, O: torch.Tensor,

@@ -193,6 +193,36 @@ int ripe_verify_attn_all_depths(ripe_cache_t cache, int layer, const int32_t* se
                                 const int32_t* ctx_len_dev, float scale, void* O, float* lse,
                                 ripe_stream_t stream);
 
+/*
+ * ripe_verify_attn for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is a deployment variant, not part of the method.
+ *
+ * Some callers cannot call cudaMalloc: a serving stack that has reserved nearly
+ * all of HBM for its own pools and forbids other allocations, code that enqueues
+ * work while a stream is being captured into a CUDA graph, or a latency-bound
+ * path that cannot afford cudaMalloc's implicit device synchronisation.  This
+ * entry point takes the same arguments and computes the same result as
+ * ripe_verify_attn, but never allocates: its per-split partial results go to a
+ * fixed device array of RIPE_NOALLOC_SCRATCH_BYTES owned by the library, which
+ * every GPU that loads the library's device code holds until the process exits.
+ *   - The first call on each device looks up that array's device address
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture on the device.
+ *   - A call whose partial results would not fit even with the deep region in
+ *     one split returns RIPE_ERR_CAPACITY (ripe_last_error gives the bytes
+ *     needed); *scratch_needed (if not NULL) receives the bytes the call uses or
+ *     would need.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it has to start at zero: each call writes every partial it
+ *     later reads.  Calls that may overlap on the GPU (different streams without
+ *     ordering between them) race on the array: serialise them.
+ */
+#define RIPE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int ripe_verify_attn_noalloc(ripe_cache_t cache, int layer, const ripe_branch_t* branches_dev, int nbranch,
+                             int nrows, const void* Q, const void* Kblk, const void* Vblk,
+                             const int32_t* ctx_len_dev, float scale, void* O, float* lse,
+                             ripe_stream_t stream, size_t* scratch_needed);
+
 /* Pre-size the verify scratch for calls with up to max_rows rows (before stream capture). */
 int ripe_reserve_workspace(ripe_cache_t cache, int max_rows);
 
