@@ -22,6 +22,11 @@ struct ripe_cache_s {
     // Verify scratch (per-split partial results), grown on demand.
     void* work;
     size_t work_bytes;
+    // TMA descriptors (CUtensorMap) of the deep K and V planes, when the tensor-core
+    // deep kernel serves this cache (bf16, d in {64, 96, 128}).
+    alignas(64) unsigned char tmap_k[128];
+    alignas(64) unsigned char tmap_v[128];
+    bool tc_ready;
 };
 
 // Store geometry, passed by value to kernels.

@@ -24,10 +24,18 @@ struct VerifyPlan {
     int nrowchunks;    // row chunks per branch
     int max_ntok;      // host bound on tokens per branch
     bool tc_deep;      // deep region on the tcgen05 stacked-query kernel
+    int mt;            // M tiles (of 128 rows) per deep CTA
+    int gslots;        // deep CTAs along the sequence-group axis
     size_t work_bytes; // scratch needed
 };
 
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths);
+
+struct VerifyArgs;
+bool deep_tc_supported(int dtype, int d);
+cudaError_t launch_deep_tc(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt,
+                           cudaStream_t st);
+int make_deep_tensor_maps(ripe_cache_s* c);
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
                           const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,

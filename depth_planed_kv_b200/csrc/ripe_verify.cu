@@ -250,24 +250,42 @@ cudaError_t launch_split(const VerifyArgs& a, int seg_first, int seg_count, int 
 }  // namespace
 
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths) {
-    (void)all_depths;
     VerifyPlan p{};
     p.max_ntok = max_ntok;
     p.rows_chunk = kRowsPerCta;
     p.nrowchunks = (max_ntok + kRowsPerCta - 1) / kRowsPerCta;
     if (p.nrowchunks < 1) p.nrowchunks = 1;
     const int A_ub = c->len_ub < c->Tmax ? c->len_ub : c->Tmax;
-    const int64_t items = (int64_t)nbranch * p.nrowchunks * c->H;
-    const int64_t target = 148 * 8;
-    int64_t ns = items > 0 ? (target + items - 1) / items : 1;
-    const int64_t max_ns = (A_ub + 63) / 64;
-    if (ns > max_ns) ns = max_ns;
-    if (ns < 1) ns = 1;
-    p.nsplit = (int)ns;
-    int chunk = (int)((A_ub + ns - 1) / ns);
-    chunk = (chunk + 31) / 32 * 32;
-    p.chunk = chunk < 32 ? 32 : chunk;
-    p.tc_deep = false;
+    p.tc_deep = c->tc_ready && deep_tc_supported(c->dtype, c->d);
+    int64_t ns;
+    if (p.tc_deep) {
+        // One deep CTA per (sequence group, head, split); splits only until the
+        // CTAs cover the 148 SMs once (each CTA holds one SM's tensor memory).
+        p.gslots = all_depths ? nbranch / c->R : (nbranch < c->Bmax ? nbranch : c->Bmax);
+        p.mt = (all_depths && max_ntok * c->R > 128) ? 2 : 1;
+        const int64_t units = (int64_t)p.gslots * c->H;
+        ns = units > 0 ? 148 / units : 1;
+        const int64_t max_ns = (A_ub + 255) / 256;
+        if (ns > max_ns) ns = max_ns;
+        if (ns < 1) ns = 1;
+        p.nsplit = (int)ns;
+        int chunk = (int)((A_ub + ns - 1) / ns);
+        chunk = (chunk + 63) / 64 * 64;
+        p.chunk = chunk < 64 ? 64 : chunk;
+    } else {
+        const int64_t items = (int64_t)nbranch * p.nrowchunks * c->H;
+        const int64_t target = 148 * 8;
+        ns = items > 0 ? (target + items - 1) / items : 1;
+        const int64_t max_ns = (A_ub + 63) / 64;
+        if (ns > max_ns) ns = max_ns;
+        if (ns < 1) ns = 1;
+        p.nsplit = (int)ns;
+        int chunk = (int)((A_ub + ns - 1) / ns);
+        chunk = (chunk + 31) / 32 * 32;
+        p.chunk = chunk < 32 ? 32 : chunk;
+        p.mt = 0;
+        p.gslots = 0;
+    }
     p.work_bytes = verify_work_bytes(nrows, c->H, c->d, p.nsplit + 1);
     return p;
 }
@@ -288,20 +306,24 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     a.part_o = reinterpret_cast<float*>(reinterpret_cast<char*>(work) +
                                         verify_ml_bytes(ba.nrows, c->H, a.nseg));
     cudaError_t e;
-    if (c->dtype == RIPE_BF16) {
+    if (plan.tc_deep) {
+        // Deep region on the tensor cores, then the window/block split, then the merge.
+        e = launch_deep_tc(c->tmap_k, c->tmap_v, a, plan.gslots, plan.mt, st);
+        if (e != cudaSuccess) return e;
+        e = launch_split<__nv_bfloat16>(a, a.nsplit, 1, ba.nbranch, st);
+        if (e != cudaSuccess) return e;
+        merge_kernel<__nv_bfloat16><<<ba.nbranch * c->H, 128, 0, st>>>(a);
+        ripe_count_launch();
+    } else if (c->dtype == RIPE_BF16) {
         e = launch_split<__nv_bfloat16>(a, 0, a.nseg, ba.nbranch, st);
         if (e != cudaSuccess) return e;
-        if (ba.nbranch > 0) {
-            merge_kernel<__nv_bfloat16><<<ba.nbranch * c->H, 128, 0, st>>>(a);
-            ripe_count_launch();
-        }
+        merge_kernel<__nv_bfloat16><<<ba.nbranch * c->H, 128, 0, st>>>(a);
+        ripe_count_launch();
     } else {
         e = launch_split<float>(a, 0, a.nseg, ba.nbranch, st);
         if (e != cudaSuccess) return e;
-        if (ba.nbranch > 0) {
-            merge_kernel<float><<<ba.nbranch * c->H, 128, 0, st>>>(a);
-            ripe_count_launch();
-        }
+        merge_kernel<float><<<ba.nbranch * c->H, 128, 0, st>>>(a);
+        ripe_count_launch();
     }
     return cudaGetLastError();
 }

@@ -65,7 +65,9 @@ enum {
     RIPE_DEVERR_CAPACITY = 2,    /* append would pass Tmax; that sequence was skipped */
     RIPE_DEVERR_COUNT = 3,       /* an accepted count outside [0, kmax_in] */
     RIPE_DEVERR_CTX = 4,         /* ctx_len above the committed length; clamped to it */
-    RIPE_DEVERR_BRANCH = 5       /* a branch with depth outside [1,R] or rows out of range */
+    RIPE_DEVERR_BRANCH = 5,      /* a branch with depth outside [1,R], rows out of range, more tokens
+                                    than the cache's kmax, or a sequence's branches not adjacent */
+    RIPE_DEVERR_TIMEOUT = 6      /* a kernel's bounded wait expired; its outputs are incomplete */
 };
 
 /*

@@ -257,3 +257,43 @@ def test_batched_equals_one_token_at_a_time_gpu():
             assert a <= 1e-5 and rel <= 1e-5
         c2.close()
     cache.close()
+
+
+@pytest.mark.parametrize("d", [64, 96, 128])
+def test_many_rows_per_sequence_branch_list(d):
+    """More than 128 query rows for one sequence (several row tiles of the deep
+    kernel), next to a sequence with few rows."""
+    wl = S.Workload("rows", 1, 8, 3, d, 16, 60, 2, None, 0.88, 61, "bf16", 700, 60)
+    ctx = np.array([650, 130])
+    cache = make_cache(wl)
+    fill(cache, wl, ctx)
+    branches = [S.BranchSpec(0, 8, 60, 0, 0), S.BranchSpec(0, 2, 60, 1, 1), S.BranchSpec(0, 5, 37, 2, 2),
+                S.BranchSpec(1, 8, 9, 0, 0), S.BranchSpec(1, 4, 3, 1, 1)]
+    table, Q, Kb, Vb = branch_rows(wl, 0, branches, [0, 1])
+    from depth_planed_kv_b200.ripe import branch_table
+    O = torch.full(Q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full(Q.shape[:2], float("nan"), device="cuda")
+    cache.ripe_verify_attn(0, branch_table([tuple(t) for t in table]), len(table), to_dev(Q, wl),
+                           to_dev(Kb, wl), to_dev(Vb, wl), O, lse)
+    torch.cuda.synchronize()
+    ws = np.maximum(ctx - wl.W, 0)
+    views = [seq_planes(wl, 0, s, int(ctx[s]), int(ws[s])) for s in range(2)]
+    ref, ref_lse = OR.verify(views, table, Q, Kb, Vb, 1 / math.sqrt(wl.d))
+    check(O.float().cpu().numpy(), ref, wl, "many rows d=%d" % d)
+    check_lse(lse.cpu().numpy(), ref_lse)
+    assert cache.ripe_get_device_error() == 0
+    cache.close()
+
+
+def test_all_depths_more_than_256_rows():
+    """k*R = 9*32 = 288 rows per sequence and head: two 128-row M tiles per CTA
+    plus a second row tile."""
+    wl = S.Workload("k9", 1, 32, 2, 128, 32, 9, 2, 300, 0.88, 71, "bf16", 400, 9)
+    cache = make_cache(wl)
+    fill(cache, wl, [300, 211])
+    _, O, lse, _ = run_all_depths(cache, wl, 0, 2, wl.k)
+    ref, ref_lse = oracle_all_depths(wl, 0, 2, wl.k, [300, 211], [300 - 32, 211 - 32])
+    check(O, ref, wl, "k=9 all depths")
+    check_lse(lse, ref_lse)
+    assert cache.ripe_get_device_error() == 0
+    cache.close()
