@@ -31,6 +31,8 @@ namespace {
 
 constexpr int kN = 64;  // keys per tile
 constexpr int kThreads = 192;
+constexpr int kMaxGroupBranches = 64;  // branches of one sequence in one call
+constexpr int kWinRows = 16;           // rows per CTA of the window kernel (its row chunks)
 
 template <int D, int MT, int ST>
 struct DeepLayout {
@@ -46,7 +48,8 @@ struct DeepLayout {
     // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
     static constexpr int NBAR = 1 + 3 * ST + 7;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int BYTES = OFF_MISC + 64;
+    static constexpr int OFF_BT = OFF_MISC + 64;           // branch table of the group
+    static constexpr int BYTES = OFF_BT + kMaxGroupBranches * 20;
     static constexpr int SMEM = BYTES + 1024;  // alignment slack
     static constexpr uint32_t TMEM_COLS = MT == 1 ? 256 : 512;
     static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
@@ -54,7 +57,13 @@ struct DeepLayout {
 };
 
 struct GroupInfo {
-    int first, end, seq, nrows, T, A, key_begin, key_end;
+    int first, nb, seq, nrows, T, A, key_begin, key_end;
+};
+
+// One branch of the group: its rows, its offset among the group's rows, and the
+// mask of its window-kernel row chunks whose merge falls to this CTA.
+struct BranchEnt {
+    int row0, stride, ntok, off, last_mask;
 };
 
 // Warp-uniform bounded wait: every lane waits, and all lanes agree on the outcome
@@ -64,14 +73,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-// Row (of Q/O) of the group's rl-th query, branches taken in table order; -1 past the end.
-__device__ int group_row(const VerifyArgs& a, const GroupInfo& G, int rl) {
-    int off = 0;
-    for (int bi = G.first; bi < G.end; ++bi) {
-        const Branch br = load_branch(a.ba, a.s.R, a.s.Bmax, bi);
-        if (!br.ok) continue;
-        if (rl < off + br.ntok) return br.row0 + (rl - off) * br.stride;
-        off += br.ntok;
+// Row (of Q/O) of the group's rl-th query, branches in table order; -1 past the end.
+__device__ int group_row(const BranchEnt* bt, int nb, int rl, int* bidx = nullptr, int* jout = nullptr) {
+    for (int i = 0; i < nb; ++i) {
+        if (rl < bt[i].off + bt[i].ntok) {
+            const int j = rl - bt[i].off;
+            if (bidx) *bidx = i;
+            if (jout) *jout = j;
+            return bt[i].row0 + j * bt[i].stride;
+        }
     }
     return -1;
 }
@@ -121,6 +131,7 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 4);
     GroupInfo* gi = reinterpret_cast<GroupInfo*>(sm + Lay::OFF_MISC + 16);
+    BranchEnt* bt = reinterpret_cast<BranchEnt*>(sm + Lay::OFF_BT);
 
     const StoreView& s = a.s;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -168,23 +179,40 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             first = min(g * s.R, a.ba.nbranch);
             end = min(first + s.R, a.ba.nbranch);
         }
-        int seq = -1, nrows = 0;
-        for (int i = first; i < end; ++i) {
-            const Branch br = load_branch(a.ba, s.R, s.Bmax, i);
-            if (!br.ok) continue;
-            seq = br.seq;
-            nrows += br.ntok;
+        int nb = end - first;
+        if (nb > kMaxGroupBranches) {
+            if (lane == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
+            nb = 0;
+        }
+        // Branch entries loaded in parallel, row offsets by a warp prefix sum.
+        int seq = -1, base = 0;
+        for (int c0 = 0; c0 < nb; c0 += 32) {
+            const int i = c0 + lane;
+            Branch br;
+            br.ok = false;
+            if (i < nb) br = load_branch(a.ba, s.R, s.Bmax, first + i);
+            const int n = (i < nb && br.ok) ? br.ntok : 0;
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (i < nb) bt[i] = BranchEnt{br.row0, br.stride, n, base + incl - n, 0};
+            const unsigned okm = __ballot_sync(0xffffffffu, i < nb && br.ok);
+            if (seq < 0 && okm) seq = __shfl_sync(0xffffffffu, br.seq, __ffs(okm) - 1);
+            base += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) {
-            GroupInfo info{first, end, seq, nrows, 0, 0, 0, 0};
-            if (seq >= 0 && nrows > 0) {
+            GroupInfo info{first, nb, seq, base, 0, 0, 0, 0};
+            if (seq >= 0 && base > 0) {
                 info.T = context_length(s.len, a.ctx, s.err, seq, false);
                 info.A = min(s.ws[seq], info.T);
                 info.key_begin = split * a.chunk;
                 info.key_end = min(info.A, info.key_begin + a.chunk);
             }
             if (g == gridDim.x - 1 && a.ba.table && end < a.ba.nbranch)
-                set_device_error(s.err, RIPE_DEVERR_BRANCH);  // branches of a sequence not adjacent
+                set_device_error(s.err, RIPE_DEVERR_BRANCH);  // more runs of sequences than CTAs
             *gi = info;
         }
     }
@@ -292,7 +320,7 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                     // Rows of this row tile (each thread finds its own), then their Q into
                     // the swizzled K-major layout.
                     for (int mt = 0; mt < MT; ++mt) {
-                        const int row = group_row(a, G, rt * RT + mt * 128 + t);
+                        const int row = group_row(bt, G.nb, rt * RT + mt * 128 + t);
                         rows[mt] = row;
                         uint8_t* dst = sQ + mt * NCH * 8192 + t * 64;
                         const uint4* src = row >= 0
@@ -400,6 +428,7 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                                 dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
                         }
                     }
+                    __threadfence();
                     tc_fence_before();
                 }
             }
@@ -410,10 +439,79 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     if (warp == 5) tmem_dealloc(tmem, Lay::TMEM_COLS);
+
+    // ---- count this split's arrival for every (branch, window row chunk) of the
+    // group; where it is the last contributor, merge those rows.
+    if (total_it > 0 && !*abort_flag) {
+        const int ndeep = deep_splits_used(G.A, a.chunk, a.nsplit);
+        if (warp == 0) {
+            for (int i = lane; i < G.nb; i += 32) {
+                int mask = 0;
+                const int nrc = (bt[i].ntok + kWinRows - 1) / kWinRows;
+                for (int rc = 0; rc < nrc; ++rc) {
+                    int* cnt = a.cnt + ((int64_t)(G.first + i) * a.nrowchunks + rc) * s.H + h;
+                    if (atomicAdd(cnt, 1) == ndeep) {
+                        *cnt = 0;
+                        mask |= 1 << rc;
+                    }
+                }
+                bt[i].last_mask = mask;
+            }
+            __threadfence();
+        }
+        __syncthreads();
+        const int nseg = a.nseg;
+        for (int rl = threadIdx.x; rl < G.nrows; rl += kThreads) {
+            int bi = 0, j = 0;
+            const int row = group_row(bt, G.nb, rl, &bi, &j);
+            if (row < 0 || !((bt[bi].last_mask >> (j / kWinRows)) & 1)) continue;
+            const int64_t base = ((int64_t)row * s.H + h) * nseg;
+            float mls[2 * 9];
+            const int np = ndeep < 8 ? ndeep : 8;
+            float M = -INFINITY;
+            for (int sg = 0; sg <= np; ++sg) {
+                const float2 ml = __ldcg(a.part_ml + base + (sg < np ? sg : a.nsplit));
+                mls[2 * sg] = ml.x;
+                mls[2 * sg + 1] = ml.y;
+                M = fmaxf(M, ml.x);
+            }
+            float L = 0.f;
+            for (int sg = 0; sg <= np; ++sg) {
+                mls[2 * sg] = ex2(mls[2 * sg] - M);
+                L = fmaf(mls[2 * sg + 1], mls[2 * sg], L);
+            }
+            const float inv = 1.f / L;
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ((int64_t)row * s.H + h) * D;
+#pragma unroll 2
+            for (int c = 0; c < D; c += 8) {
+                float acc[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+                for (int sg = 0; sg <= np; ++sg) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        a.part_o + (base + (sg < np ? sg : a.nsplit)) * D + c);
+                    const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+                    const float f = mls[2 * sg];
+                    acc[0] = fmaf(x0.x, f, acc[0]); acc[1] = fmaf(x0.y, f, acc[1]);
+                    acc[2] = fmaf(x0.z, f, acc[2]); acc[3] = fmaf(x0.w, f, acc[3]);
+                    acc[4] = fmaf(x1.x, f, acc[4]); acc[5] = fmaf(x1.y, f, acc[5]);
+                    acc[6] = fmaf(x1.z, f, acc[6]); acc[7] = fmaf(x1.w, f, acc[7]);
+                }
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+                    w4[e] = *reinterpret_cast<uint32_t*>(&b2);
+                }
+                *reinterpret_cast<uint4*>(orow + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            if (a.lse) a.lse[(int64_t)row * s.H + h] = (M + log2f(L)) * 0.69314718055994531f;
+        }
+    }
 }
 
 template <int D, int MT, int ST>
-cudaError_t launch_deep_t(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyArgs& a, int gslots,
+cudaError_t launch_deep_t(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyArgs& a, int gslots, bool pdl,
                           cudaStream_t st) {
     using Lay = DeepLayout<D, MT, ST>;
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
@@ -422,12 +520,24 @@ cudaError_t launch_deep_t(const CUtensorMap& tk, const CUtensorMap& tv, const Ve
         cudaError_t e = cudaFuncSetAttribute(deep_kernel<D, MT, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Lay::SMEM);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(deep_kernel<D, MT, ST>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         configured = true;
     }
-    dim3 grid(gslots, a.s.H, a.nsplit);
-    deep_kernel<D, MT, ST><<<grid, kThreads, Lay::SMEM, st>>>(tk, tv, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gslots, a.s.H, a.nsplit);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Lay::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, deep_kernel<D, MT, ST>, tk, tv, a);
     ripe_count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace
@@ -436,19 +546,19 @@ bool deep_tc_supported(int dtype, int d) {
     return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128);
 }
 
-cudaError_t launch_deep_tc(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt,
+cudaError_t launch_deep_tc(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt, bool pdl,
                            cudaStream_t st) {
     const CUtensorMap& tk = *reinterpret_cast<const CUtensorMap*>(tmK);
     const CUtensorMap& tv = *reinterpret_cast<const CUtensorMap*>(tmV);
     const int d = a.s.d;
     if (mt == 1) {
-        if (d == 64) return launch_deep_t<64, 1, 4>(tk, tv, a, gslots, st);
-        if (d == 96) return launch_deep_t<96, 1, 3>(tk, tv, a, gslots, st);
-        if (d == 128) return launch_deep_t<128, 1, 3>(tk, tv, a, gslots, st);
+        if (d == 64) return launch_deep_t<64, 1, 4>(tk, tv, a, gslots, pdl, st);
+        if (d == 96) return launch_deep_t<96, 1, 3>(tk, tv, a, gslots, pdl, st);
+        if (d == 128) return launch_deep_t<128, 1, 3>(tk, tv, a, gslots, pdl, st);
     } else {
-        if (d == 64) return launch_deep_t<64, 2, 4>(tk, tv, a, gslots, st);
-        if (d == 96) return launch_deep_t<96, 2, 3>(tk, tv, a, gslots, st);
-        if (d == 128) return launch_deep_t<128, 2, 3>(tk, tv, a, gslots, st);
+        if (d == 64) return launch_deep_t<64, 2, 4>(tk, tv, a, gslots, pdl, st);
+        if (d == 96) return launch_deep_t<96, 2, 3>(tk, tv, a, gslots, pdl, st);
+        if (d == 128) return launch_deep_t<128, 2, 3>(tk, tv, a, gslots, pdl, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -51,6 +51,18 @@ cudaError_t static_scratch_address(void** out) {
 
 }  // namespace
 
+cudaError_t reset_noalloc_counters(cudaStream_t st) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return e;
+    void* p = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        p = g_scratch_addr[dev];
+    }
+    return reset_verify_counters(p, st);
+}
+
 extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_branch_t* branches, int nbranch,
                                         int nrows, const void* Q, const void* Kb, const void* Vb,
                                         const int32_t* ctx, float scale, void* O, float* lse,
@@ -73,6 +85,9 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
     ba.nrows = nrows;
     ba.max_ntok = c->kmax;
     VerifyPlan plan = plan_verify(c, nbranch, nrows, c->kmax, false);
+    if (plan.counters > verify_max_counters())
+        return ripe_fail(RIPE_ERR_CAPACITY, "%lld (branch, row chunk, head) units in one call; at most %lld",
+                         (long long)plan.counters, (long long)verify_max_counters());
     // Fewer, longer deep splits until the partial results fit the fixed array.
     while (plan.work_bytes > kStaticScratchBytes && plan.nsplit > 1) {
         plan.nsplit = plan.nsplit / 2;

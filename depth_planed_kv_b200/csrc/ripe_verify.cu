@@ -17,13 +17,13 @@
 #include "ripe_internal.cuh"
 #include "ripe_launch.h"
 #include "ripe_verify.cuh"
+#include "sm100_ptx.cuh"
 
 namespace {
 
 constexpr int kWarps = 4;
 constexpr int kRowsPerWarp = 4;
 constexpr int kRowsPerCta = kWarps * kRowsPerWarp;
-constexpr int kTile = 32;
 
 template <typename Elem>
 __device__ inline float to_f32(Elem x);
@@ -50,19 +50,38 @@ __device__ inline float warp_sum(float v) {
     return v;
 }
 
-// One CTA: up to 16 rows of one branch, one head, one split.  Keys stream
-// through shared memory 32 at a time; each warp owns 4 rows; a lane owns one
-// key for the scores and d/32 output channels for the weighted sum.
+// One CTA: up to 16 rows of one branch, one head, one split of its keys.
+//
+// The split's keys (a contiguous run of the deep plane, or the window run of
+// plane r -- the ring, which wraps at most once -- followed by the branch's
+// draft-block tokens) stream into shared memory in tiles of KT keys by bulk
+// asynchronous copies (one or two stages).  Per tile:
+//   A. scores: thread = key; each K row is read once for all rows, 16 bytes at a
+//      time with a per-key rotation of the starting vector (no bank conflicts
+//      for any head size);
+//   B. softmax: warp = row; tile max, rescale factor, probabilities in place;
+//   C. P.V: warp = row group, lane = output channel; each V row read once per
+//      warp for all of its rows.
+// The split's partial (m, l, o) of every row goes to the scratch.
 template <typename Elem, int MAXD>
 __global__ void __launch_bounds__(kWarps * 32)
-split_kernel(VerifyArgs a, int seg_first, int seg_count) {
+seg_kernel(VerifyArgs a, int seg_first, int seg_count, int KT, int ST) {
+    using namespace sm100;
     constexpr int NV = MAXD / 32;
-    __shared__ float q_s[kRowsPerCta][MAXD];
-    __shared__ float k_s[kTile][MAXD + 1];
-    __shared__ float v_s[kTile][MAXD];
+    constexpr int VE = 16 / sizeof(Elem);  // elements per 16-byte vector
+    extern __shared__ __align__(128) uint8_t smem[];
 
     const StoreView& s = a.s;
     const int d = s.d, H = s.H;
+    const int rowb = d * (int)sizeof(Elem);  // bytes per key row
+    const int nvec = rowb / 16;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16);
+    uint8_t* sK = smem + 128;
+    uint8_t* sV = sK + (size_t)ST * KT * rowb;
+    float* q_s = reinterpret_cast<float*>(sV + (size_t)ST * KT * rowb);
+    float* sc = q_s + kRowsPerCta * d;
+
     int w = blockIdx.x;
     const int seg = seg_first + w % seg_count; w /= seg_count;
     const int h = w % H; w /= H;
@@ -80,12 +99,11 @@ split_kernel(VerifyArgs a, int seg_first, int seg_count) {
     const int T = context_length(s.len, a.ctx, s.err, b, seg == a.nsplit && h == 0 && rc == 0 && threadIdx.x == 0);
     const int A = min(s.ws[b], T);
 
-    int64_t p0, p1;
-    int nblk = 0;
+    int p0, p1, nblk = 0;
     bool ring = false;
     if (seg < a.nsplit) {
-        p0 = (int64_t)seg * a.chunk;
-        p1 = min((int64_t)A, p0 + a.chunk);
+        p0 = seg * a.chunk;
+        p1 = min(A, p0 + a.chunk);
         if (p0 >= p1) return;
     } else {
         p0 = A;
@@ -93,101 +111,184 @@ split_kernel(VerifyArgs a, int seg_first, int seg_count) {
         nblk = j0 + nr;  // block tokens 0..j0+nr-1 are visible to some row here
         ring = r < s.R;
     }
-    const int ncom = (int)(p1 - p0);
+    const int ncom = p1 - p0;
     const int nk = ncom + nblk;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int ntile = (nk + KT - 1) / KT;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
-    for (int e = threadIdx.x; e < nr * d; e += blockDim.x) {
+    if (tid == 0) {
+        for (int i = 0; i < ST; ++i) mbar_init(full + i, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // Issue the copies of tile t into stage t % ST (one thread).
+    auto issue_tile = [&](int t) {
+        const int st = t % ST;
+        const int k0 = t * KT, k1 = min(nk, k0 + KT);
+        uint8_t* dk = sK + (size_t)st * KT * rowb;
+        uint8_t* dv = sV + (size_t)st * KT * rowb;
+        mbar_expect_tx(full + st, (uint32_t)(2 * (k1 - k0) * rowb));
+        int key = k0;
+        while (key < min(k1, ncom)) {
+            const int p = p0 + key;
+            int n = min(k1, ncom) - key;
+            int64_t off;
+            const char *kb, *vb;
+            if (ring) {
+                const int slot = p % s.Wcap;
+                n = min(n, s.Wcap - slot);
+                off = ring_row(s, a.layer, b, h, r, slot);
+                kb = s.kwin; vb = s.vwin;
+            } else {
+                off = deep_row(s, a.layer, b, h, p);
+                kb = s.kdeep; vb = s.vdeep;
+            }
+            bulk_load(dk + (size_t)(key - k0) * rowb, kb + off, (uint32_t)(n * rowb), full + st);
+            bulk_load(dv + (size_t)(key - k0) * rowb, vb + off, (uint32_t)(n * rowb), full + st);
+            key += n;
+        }
+        for (; key < k1; ++key) {
+            const int64_t row = br.row0 + (int64_t)(key - ncom) * br.stride;
+            const int64_t off = (row * H + h) * rowb;
+            bulk_load(dk + (size_t)(key - k0) * rowb, a.Kb + off, (uint32_t)rowb, full + st);
+            bulk_load(dv + (size_t)(key - k0) * rowb, a.Vb + off, (uint32_t)rowb, full + st);
+        }
+    };
+    if (tid == 0) {
+        for (int t = 0; t < ST && t < ntile; ++t) issue_tile(t);
+    }
+
+    for (int e = tid; e < nr * d; e += blockDim.x) {
         const int rr = e / d, c = e % d;
         const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
-        q_s[rr][c] = to_f32(reinterpret_cast<const Elem*>(a.Q)[(row * H + h) * d + c]) * a.scale_log2;
+        q_s[rr * d + c] = to_f32(reinterpret_cast<const Elem*>(a.Q)[(row * H + h) * d + c]) * a.scale_log2;
     }
 
     float m[kRowsPerWarp], l[kRowsPerWarp], o[kRowsPerWarp][NV];
 #pragma unroll
-    for (int t = 0; t < kRowsPerWarp; ++t) {
-        m[t] = -INFINITY;
-        l[t] = 0.f;
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        m[i] = -INFINITY;
+        l[i] = 0.f;
 #pragma unroll
-        for (int v = 0; v < NV; ++v) o[t][v] = 0.f;
+        for (int v = 0; v < NV; ++v) o[i][v] = 0.f;
     }
 
-    for (int k0 = 0; k0 < nk; k0 += kTile) {
-        __syncthreads();
-        for (int e = threadIdx.x; e < kTile * d; e += blockDim.x) {
-            const int key = e / d, c = e % d;
-            const int t = k0 + key;
-            float kx = 0.f, vx = 0.f;
-            if (t < nk) {
-                const Elem *kp, *vp;
-                if (t < ncom) {
-                    const int64_t p = p0 + t;
-                    if (ring) {
-                        const int64_t off = ring_row(s, a.layer, b, h, r, (int)(p % s.Wcap));
-                        kp = reinterpret_cast<const Elem*>(s.kwin + off);
-                        vp = reinterpret_cast<const Elem*>(s.vwin + off);
-                    } else {
-                        const int64_t off = deep_row(s, a.layer, b, h, p);
-                        kp = reinterpret_cast<const Elem*>(s.kdeep + off);
-                        vp = reinterpret_cast<const Elem*>(s.vdeep + off);
+    for (int t = 0; t < ntile; ++t) {
+        const int st = t % ST;
+        const int k0 = t * KT, nkt = min(nk, k0 + KT) - k0;
+        mbar_wait(full + st, (t / ST) & 1, abort_flag, s.err);
+        __syncthreads();  // q_s written; a timed-out wait still keeps every thread in step
+        const uint8_t* tk = sK + (size_t)st * KT * rowb;
+        const uint8_t* tv = sV + (size_t)st * KT * rowb;
+        // A. scores (log2 units): thread = key
+        for (int kk = tid; kk < nkt; kk += blockDim.x) {
+            float acc[kRowsPerCta];
+#pragma unroll
+            for (int rr = 0; rr < kRowsPerCta; ++rr) acc[rr] = 0.f;
+            const uint4* krow = reinterpret_cast<const uint4*>(tk + (size_t)kk * rowb);
+            for (int v = 0; v < nvec; ++v) {
+                int vv = v + kk;
+                vv -= (vv / nvec) * nvec;
+                const uint4 x = krow[vv];
+                float kf[VE];
+                if constexpr (sizeof(Elem) == 2) {
+                    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(b2[e]);
+                        kf[2 * e] = f.x;
+                        kf[2 * e + 1] = f.y;
                     }
                 } else {
-                    const int64_t row = br.row0 + (int64_t)(t - ncom) * br.stride;
-                    kp = reinterpret_cast<const Elem*>(a.Kb) + (row * H + h) * d;
-                    vp = reinterpret_cast<const Elem*>(a.Vb) + (row * H + h) * d;
+                    kf[0] = __uint_as_float(x.x); kf[1] = __uint_as_float(x.y);
+                    kf[2] = __uint_as_float(x.z); kf[3] = __uint_as_float(x.w);
                 }
-                kx = to_f32(kp[c]);
-                vx = to_f32(vp[c]);
+#pragma unroll
+                for (int rr = 0; rr < kRowsPerCta; ++rr) {
+                    if (rr < nr) {
+                        const float* qv = q_s + rr * d + vv * VE;
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) acc[rr] = fmaf(qv[e], kf[e], acc[rr]);
+                    }
+                }
             }
-            k_s[key][c] = kx;
-            v_s[key][c] = vx;
+            const int key = k0 + kk;
+#pragma unroll
+            for (int rr = 0; rr < kRowsPerCta; ++rr) {
+                if (rr < nr) {
+                    const bool masked = key >= ncom && key - ncom > j0 + rr;
+                    sc[rr * KT + kk] = masked ? -INFINITY : acc[rr];
+                }
+            }
         }
         __syncthreads();
-        const int t = k0 + lane;
+        // B. online softmax: warp = row
+        float alpha[kRowsPerWarp];
 #pragma unroll
-        for (int rw = 0; rw < kRowsPerWarp; ++rw) {
-            const int rr = warp + kWarps * rw;
-            if (rr >= nr) break;
-            const int j = j0 + rr;
-            const bool valid = t < nk && (t < ncom || (t - ncom) <= j);
-            float sc = -INFINITY;
-            if (valid) {
-                float acc = 0.f;
-                for (int c = 0; c < d; ++c) acc = fmaf(q_s[rr][c], k_s[lane][c], acc);
-                sc = acc;
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            alpha[i] = 1.f;
+            const int rr = warp + kWarps * i;
+            if (rr >= nr) continue;
+            float* srow = sc + rr * KT;
+            float mt = -INFINITY;
+            for (int kk = lane; kk < nkt; kk += 32) mt = fmaxf(mt, srow[kk]);
+            mt = warp_max(mt);
+            const float mn = fmaxf(m[i], mt);
+            if (mn == -INFINITY) {
+                for (int kk = lane; kk < nkt; kk += 32) srow[kk] = 0.f;
+                continue;
             }
-            const float mt = warp_max(sc);
-            const float mn = fmaxf(m[rw], mt);
-            if (mn == -INFINITY) continue;
-            const float alpha = exp2f(m[rw] - mn);
-            const float p = valid ? exp2f(sc - mn) : 0.f;
-            l[rw] = l[rw] * alpha + warp_sum(p);
-            m[rw] = mn;
+            alpha[i] = ex2(m[i] - mn);
+            float sum = 0.f;
+            for (int kk = lane; kk < nkt; kk += 32) {
+                const float p = ex2(srow[kk] - mn);
+                srow[kk] = p;
+                sum += p;
+            }
+            l[i] = l[i] * alpha[i] + warp_sum(sum);
+            m[i] = mn;
+        }
+        __syncwarp();
+        // C. o = alpha*o + P V: warp = its rows, lane = channels
 #pragma unroll
-            for (int v = 0; v < NV; ++v) o[rw][v] *= alpha;
-            const int kmax = min(kTile, nk - k0);
-            for (int key = 0; key < kmax; ++key) {
-                const float pk = __shfl_sync(0xffffffffu, p, key);
+        for (int i = 0; i < kRowsPerWarp; ++i)
 #pragma unroll
-                for (int v = 0; v < NV; ++v) {
-                    const int c = lane + 32 * v;
-                    if (c < d) o[rw][v] = fmaf(pk, v_s[key][c], o[rw][v]);
+            for (int v = 0; v < NV; ++v) o[i][v] *= alpha[i];
+        const int nrw = nr > warp ? (nr - warp + kWarps - 1) / kWarps : 0;
+        for (int kk = 0; kk < nkt; ++kk) {
+            const Elem* vrow = reinterpret_cast<const Elem*>(tv + (size_t)kk * rowb);
+            float vv[NV];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const int c = lane + 32 * v;
+                vv[v] = c < d ? to_f32(vrow[c]) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < kRowsPerWarp; ++i) {
+                if (i < nrw) {
+                    const float p = sc[(warp + kWarps * i) * KT + kk];
+#pragma unroll
+                    for (int v = 0; v < NV; ++v) o[i][v] = fmaf(p, vv[v], o[i][v]);
                 }
             }
         }
+        __syncthreads();
+        if (tid == 0 && t + ST < ntile) issue_tile(t + ST);
     }
 
 #pragma unroll
-    for (int rw = 0; rw < kRowsPerWarp; ++rw) {
-        const int rr = warp + kWarps * rw;
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int rr = warp + kWarps * i;
         if (rr >= nr) break;
         const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
         const int64_t pi = (row * H + h) * a.nseg + seg;
-        if (lane == 0) a.part_ml[pi] = make_float2(m[rw], l[rw]);
+        if (lane == 0) a.part_ml[pi] = make_float2(m[i], l[i]);
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
             const int c = lane + 32 * v;
-            if (c < d) a.part_o[pi * d + c] = o[rw][v];
+            if (c < d) a.part_o[pi * d + c] = o[i][v];
         }
     }
 }
@@ -234,15 +335,57 @@ __global__ void __launch_bounds__(128) merge_kernel(VerifyArgs a) {
     }
 }
 
+// Key tile and stage count of the CUDA-core kernel: one stage when a split's keys
+// fit a tile of at most 128, else two stages of 128-key tiles.
+struct SegShape {
+    int KT, ST;
+    size_t smem;
+};
+
+SegShape seg_shape(int d, int esize, int keys_ub) {
+    SegShape g;
+    if (keys_ub <= 128) {
+        g.KT = (keys_ub + 7) / 8 * 8;
+        if (g.KT < 8) g.KT = 8;
+        g.ST = 1;
+    } else {
+        g.KT = 128;
+        g.ST = 2;
+    }
+    auto bytes = [&](int KT, int ST) {
+        return 128 + (size_t)2 * ST * KT * d * esize + (size_t)kRowsPerCta * d * 4 + (size_t)kRowsPerCta * KT * 4;
+    };
+    while (bytes(g.KT, g.ST) > 150 * 1024 && g.KT > 16) g.KT = (g.KT / 2 + 7) / 8 * 8;
+    g.smem = bytes(g.KT, g.ST);
+    return g;
+}
+
 template <typename Elem>
-cudaError_t launch_split(const VerifyArgs& a, int seg_first, int seg_count, int nbranch, cudaStream_t st) {
+cudaError_t launch_seg(const VerifyArgs& a, int seg_first, int seg_count, int nbranch, int keys_ub,
+                       cudaStream_t st) {
     const int64_t grid = (int64_t)nbranch * a.nrowchunks * a.s.H * seg_count;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    if (a.s.d <= 64)
-        split_kernel<Elem, 64><<<(unsigned)grid, kWarps * 32, 0, st>>>(a, seg_first, seg_count);
-    else
-        split_kernel<Elem, 128><<<(unsigned)grid, kWarps * 32, 0, st>>>(a, seg_first, seg_count);
+    const SegShape g = seg_shape(a.s.d, (int)sizeof(Elem), keys_ub);
+    if (a.s.d <= 64) {
+        static bool cfg = false;
+        if (!cfg) {
+            cudaFuncSetAttribute(seg_kernel<Elem, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+            cudaFuncSetAttribute(seg_kernel<Elem, 64>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cfg = true;
+        }
+        seg_kernel<Elem, 64><<<(unsigned)grid, kWarps * 32, g.smem, st>>>(a, seg_first, seg_count, g.KT, g.ST);
+    } else {
+        static bool cfg = false;
+        if (!cfg) {
+            cudaFuncSetAttribute(seg_kernel<Elem, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+            cudaFuncSetAttribute(seg_kernel<Elem, 128>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cfg = true;
+        }
+        seg_kernel<Elem, 128><<<(unsigned)grid, kWarps * 32, g.smem, st>>>(a, seg_first, seg_count, g.KT, g.ST);
+    }
     ripe_count_launch();
     return cudaGetLastError();
 }
@@ -265,7 +408,8 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
         p.mt = (all_depths && max_ntok * c->R > 128) ? 2 : 1;
         const int64_t units = (int64_t)p.gslots * c->H;
         ns = units > 0 ? 148 / units : 1;
-        const int64_t max_ns = (A_ub + 255) / 256;
+        int64_t max_ns = (A_ub + 255) / 256;
+        if (max_ns > 8) max_ns = 8;  // the deep-side merge combines at most 8 deep partials
         if (ns > max_ns) ns = max_ns;
         if (ns < 1) ns = 1;
         p.nsplit = (int)ns;
@@ -287,7 +431,14 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
         p.gslots = 0;
     }
     p.work_bytes = verify_work_bytes(nrows, c->H, c->d, p.nsplit + 1);
+    p.counters = (int64_t)nbranch * p.nrowchunks * c->H;
     return p;
+}
+
+int64_t verify_max_counters() { return kMaxCounters; }
+
+cudaError_t reset_verify_counters(void* work, cudaStream_t st) {
+    return work ? cudaMemsetAsync(work, 0, kCounterBytes, st) : cudaSuccess;
 }
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
@@ -302,27 +453,31 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     a.scale_log2 = scale * 1.4426950408889634f;
     a.nsplit = plan.nsplit; a.chunk = plan.chunk; a.nseg = plan.nsplit + 1;
     a.nrowchunks = plan.nrowchunks;
-    a.part_ml = reinterpret_cast<float2*>(work);
-    a.part_o = reinterpret_cast<float*>(reinterpret_cast<char*>(work) +
-                                        verify_ml_bytes(ba.nrows, c->H, a.nseg));
+    char* wb = reinterpret_cast<char*>(work);
+    a.cnt = reinterpret_cast<int*>(wb);
+    a.done = reinterpret_cast<int*>(wb + kCounterBytes - 256);
+    a.part_ml = reinterpret_cast<float2*>(wb + kCounterBytes);
+    a.part_o = reinterpret_cast<float*>(wb + kCounterBytes + verify_ml_bytes(ba.nrows, c->H, a.nseg));
     cudaError_t e;
+    const int win_ub = (c->len_ub < c->Wcap ? c->len_ub : c->Wcap) + plan.max_ntok;
     if (plan.tc_deep) {
-        // Deep region on the tensor cores, then the window/block split, then the merge.
-        e = launch_deep_tc(c->tmap_k, c->tmap_v, a, plan.gslots, plan.mt, st);
+        // Deep region on the tensor cores and, beside it (programmatic dependent
+        // launch), the window/block kernel; the last contributor of a row merges.
+        e = launch_deep_tc(c->tmap_k, c->tmap_v, a, plan.gslots, plan.mt, true, st);
         if (e != cudaSuccess) return e;
-        e = launch_split<__nv_bfloat16>(a, a.nsplit, 1, ba.nbranch, st);
+        e = launch_window(a, ba.nbranch, win_ub, true, st);
         if (e != cudaSuccess) return e;
-        merge_kernel<__nv_bfloat16><<<ba.nbranch * c->H, 128, 0, st>>>(a);
-        ripe_count_launch();
-    } else if (c->dtype == RIPE_BF16) {
-        e = launch_split<__nv_bfloat16>(a, 0, a.nseg, ba.nbranch, st);
-        if (e != cudaSuccess) return e;
-        merge_kernel<__nv_bfloat16><<<ba.nbranch * c->H, 128, 0, st>>>(a);
-        ripe_count_launch();
     } else {
-        e = launch_split<float>(a, 0, a.nseg, ba.nbranch, st);
-        if (e != cudaSuccess) return e;
-        merge_kernel<float><<<ba.nbranch * c->H, 128, 0, st>>>(a);
+        const int keys_ub = plan.chunk > win_ub ? plan.chunk : win_ub;
+        if (c->dtype == RIPE_BF16) {
+            e = launch_seg<__nv_bfloat16>(a, 0, a.nseg, ba.nbranch, keys_ub, st);
+            if (e != cudaSuccess) return e;
+            merge_kernel<__nv_bfloat16><<<ba.nbranch * c->H, 128, 0, st>>>(a);
+        } else {
+            e = launch_seg<float>(a, 0, a.nseg, ba.nbranch, keys_ub, st);
+            if (e != cudaSuccess) return e;
+            merge_kernel<float><<<ba.nbranch * c->H, 128, 0, st>>>(a);
+        }
         ripe_count_launch();
     }
     return cudaGetLastError();

@@ -1,0 +1,358 @@
+// ripe_window.cu -- the window planes and the draft block of RIPE verify-attention
+// on CUDA cores, and the final merge of each row's partial results.
+//
+// A query at loop depth r reads plane r of the positions still inside the window
+// (RIPE abstract, sentence introducing RIPE) and the draft-block tokens of its own
+// branch at plane r.  Those keys differ from depth to depth, so there is nothing
+// to stack across rows: one CTA takes the k (<= 16) rows of one branch and head,
+// and the work is 4-16 dot products per key -- CUDA-core territory.
+//
+// Data movement: the CTA's keys (a run of ring slots that wraps at most once, or a
+// run of the deep plane for rows at depth R, then the block tokens) arrive by
+// 16-byte asynchronous copies spread over all threads: K rows land at a padded
+// stride (an odd number of 16-byte units, so one 16-byte vector per lane hits
+// distinct banks), V rows densely.  (Bulk copies of single 192-byte rows were
+// tried first: the copy engine then becomes the bottleneck.)
+// Compute per tile: scores with thread = key (K row read once, q broadcast from
+// shared memory), the online softmax with warp = row, P.V with thread = channel.
+//
+// Merge: the window CTA and the deep CTAs of the same (branch, row chunk, head)
+// each write a partial (m, l, o) and then count their arrival; whoever arrives
+// last merges -- M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L -- and
+// writes O and the LSE.  No one waits for anyone.
+#include "ripe_launch.h"
+#include "ripe_verify.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kRowChunk = 16;  // rows of a branch per window CTA (the launch's row chunks)
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <int D, int NR>
+struct WinLayout {
+    static constexpr int ROWB = D * 2;       // bf16 row
+    static constexpr int KSTR = ROWB + 16;   // padded K row stride: odd number of 16-byte units
+    static constexpr int NVEC = ROWB / 16;
+    // K tile, V tile, q rows (fp32), scores [row][key], probabilities [key][row], (m, l) per row
+    static size_t bytes(int KT) {
+        return 128 + (size_t)KT * (KSTR + ROWB) + (size_t)NR * D * 4 + (size_t)2 * NR * KT * 4 + NR * 8;
+    }
+};
+
+// NR = rows per CTA (4, 8 or 16): every row loop has a compile-time trip count.
+template <int D, int NR>
+__global__ void __launch_bounds__(kThreads) window_kernel(VerifyArgs a, int KT) {
+    using namespace sm100;
+    using Lay = WinLayout<D, NR>;
+    constexpr int kRows = NR;
+    constexpr int ROWB = Lay::ROWB, KSTR = Lay::KSTR, NVEC = Lay::NVEC;
+    extern __shared__ __align__(128) uint8_t smem[];
+    int* flags = reinterpret_cast<int*>(smem + 8);  // [0] merge here, [1] abort
+    uint8_t* sK = smem + 128;
+    uint8_t* sV = sK + (size_t)KT * KSTR;
+    float* q_s = reinterpret_cast<float*>(sV + (size_t)KT * ROWB);
+    float* sc = q_s + kRows * D;                // scores, [row][key]
+    float* pt = sc + (size_t)kRows * KT;        // probabilities, [key][row]
+    float* alph = pt + (size_t)kRows * KT;
+
+    const StoreView& s = a.s;
+    const int H = s.H;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    int w = blockIdx.x;
+    const int h = w % H; w /= H;
+    const int rc = w % a.nrowchunks;
+    const int bi = w / a.nrowchunks;
+
+    const Branch br = load_branch(a.ba, s.R, s.Bmax, bi);
+    if (!br.ok && tid == 0 && rc == 0 && h == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
+    const int j0 = rc * kRowChunk;
+    const bool active = br.ok && j0 < br.ntok;
+
+    if (active) {
+        const int nr = min(kRows, br.ntok - j0);
+        const int b = br.seq, r = br.depth;
+        const int T = context_length(s.len, a.ctx, s.err, b, h == 0 && rc == 0 && tid == 0);
+        const int A = min(s.ws[b], T);
+        const int nwin = T - A;
+        const int nk = nwin + j0 + nr;  // block tokens 0..j0+nr-1 are visible to some row here
+        const bool ring = r < s.R;
+        const int ntile = (nk + KT - 1) / KT;
+        const int slot0 = A % s.Wcap;  // ring slot of the first window position
+        const int64_t ring_base = ring ? ring_row(s, a.layer, b, h, r, 0) : 0;
+        if (tid == 0) flags[1] = 0;
+        for (int e = tid; e < kRows * D; e += kThreads) {
+            const int rr = e / D, c = e % D;
+            float qv = 0.f;
+            if (rr < nr) {
+                const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
+                qv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.Q)[(row * H + h) * D + c]) *
+                     a.scale_log2;
+            }
+            q_s[rr * D + c] = qv;
+        }
+        __syncthreads();
+
+        float mrow[kRows / 4], lrow[kRows / 4];  // warp w: rows w, w+4, w+8, w+12
+#pragma unroll
+        for (int i = 0; i < kRows / 4; ++i) { mrow[i] = -INFINITY; lrow[i] = 0.f; }
+        float o[kRows];
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) o[i] = 0.f;
+
+        for (int t = 0; t < ntile; ++t) {
+            const int k0 = t * KT, nkt = min(nk - k0, KT);
+            // All threads: 16-byte asynchronous copies of the tile's K rows (padded
+            // stride) and V rows (dense); consecutive threads take consecutive 16-byte
+            // pieces of a row, so each run of key rows is read coalesced.
+            for (int e = tid; e < nkt * NVEC; e += kThreads) {
+                const int kk = e / NVEC, v = e - kk * NVEC;
+                const int key = k0 + kk;
+                const char *ks, *vs;
+                if (key < nwin) {
+                    const int p = A + key;
+                    int64_t off;
+                    if (ring) {
+                        int slot = slot0 + key;
+                        if (slot >= s.Wcap) slot -= s.Wcap;
+                        off = ring_base + (int64_t)slot * ROWB;
+                        ks = s.kwin + off; vs = s.vwin + off;
+                    } else {
+                        off = deep_row(s, a.layer, b, h, p);
+                        ks = s.kdeep + off; vs = s.vdeep + off;
+                    }
+                } else {
+                    const int64_t row = br.row0 + (int64_t)(key - nwin) * br.stride;
+                    const int64_t off = (row * H + h) * ROWB;
+                    ks = a.Kb + off; vs = a.Vb + off;
+                }
+                cp_async16(sK + (size_t)kk * KSTR + 16 * v, ks + 16 * v);
+                cp_async16(sV + (size_t)kk * ROWB + 16 * v, vs + 16 * v);
+            }
+            cp_async_commit();
+            cp_async_wait_all();
+            __syncthreads();
+            // A. scores in log2 units: thread = key; q rows broadcast from shared memory
+            for (int kk = tid; kk < nkt; kk += kThreads) {
+                float acc[kRows];
+#pragma unroll
+                for (int rr = 0; rr < kRows; ++rr) acc[rr] = 0.f;
+                const uint4* krow = reinterpret_cast<const uint4*>(sK + (size_t)kk * KSTR);
+#pragma unroll 2
+                for (int v = 0; v < NVEC; ++v) {
+                    const uint4 x = krow[v];
+                    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                    float kf[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        kf[2 * e] = __uint_as_float(xw[e] << 16);
+                        kf[2 * e + 1] = __uint_as_float(xw[e] & 0xFFFF0000u);
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < kRows; ++rr) {
+                        const float4 qa = *reinterpret_cast<const float4*>(q_s + rr * D + 8 * v);
+                        const float4 qb = *reinterpret_cast<const float4*>(q_s + rr * D + 8 * v + 4);
+                        acc[rr] = fmaf(qa.x, kf[0], acc[rr]);
+                        acc[rr] = fmaf(qa.y, kf[1], acc[rr]);
+                        acc[rr] = fmaf(qa.z, kf[2], acc[rr]);
+                        acc[rr] = fmaf(qa.w, kf[3], acc[rr]);
+                        acc[rr] = fmaf(qb.x, kf[4], acc[rr]);
+                        acc[rr] = fmaf(qb.y, kf[5], acc[rr]);
+                        acc[rr] = fmaf(qb.z, kf[6], acc[rr]);
+                        acc[rr] = fmaf(qb.w, kf[7], acc[rr]);
+                    }
+                }
+                const int key = k0 + kk;
+#pragma unroll
+                for (int rr = 0; rr < kRows; ++rr) {
+                    const bool masked = rr >= nr || (key >= nwin && key - nwin > j0 + rr);
+                    sc[rr * KT + kk] = masked ? -INFINITY : acc[rr];
+                }
+            }
+            __syncthreads();
+            // B. online softmax: warp = row; probabilities go to pt[key][row]
+#pragma unroll
+            for (int i = 0; i < kRows / 4; ++i) {
+                const int rr = warp + 4 * i;
+                const float* srow = sc + (size_t)rr * KT;
+                float mt = -INFINITY;
+                for (int kk = lane; kk < nkt; kk += 32) mt = fmaxf(mt, srow[kk]);
+                mt = warp_max(mt);
+                const float mn = fmaxf(mrow[i], mt);
+                float alpha = 1.f;
+                if (mn == -INFINITY) {
+                    for (int kk = lane; kk < nkt; kk += 32) pt[kk * kRows + rr] = 0.f;
+                } else {
+                    alpha = ex2(mrow[i] - mn);
+                    float sum = 0.f;
+                    for (int kk = lane; kk < nkt; kk += 32) {
+                        const float p = ex2(srow[kk] - mn);
+                        pt[kk * kRows + rr] = p;
+                        sum += p;
+                    }
+                    lrow[i] = lrow[i] * alpha + warp_sum(sum);
+                    mrow[i] = mn;
+                }
+                if (lane == 0) alph[rr] = alpha;
+            }
+            __syncthreads();
+            // C. o = alpha*o + P V: thread = channel, all rows
+            if (tid < D) {
+#pragma unroll
+                for (int rr = 0; rr < kRows; ++rr) o[rr] *= alph[rr];
+                const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(sV) + tid;
+#pragma unroll 4
+                for (int kk = 0; kk < nkt; ++kk) {
+                    const float v = __bfloat162float(vcol[(size_t)kk * D]);
+                    const float4* pk = reinterpret_cast<const float4*>(pt + kk * kRows);
+#pragma unroll
+                    for (int q4 = 0; q4 < kRows / 4; ++q4) {
+                        const float4 p = pk[q4];
+                        o[4 * q4] = fmaf(p.x, v, o[4 * q4]);
+                        o[4 * q4 + 1] = fmaf(p.y, v, o[4 * q4 + 1]);
+                        o[4 * q4 + 2] = fmaf(p.z, v, o[4 * q4 + 2]);
+                        o[4 * q4 + 3] = fmaf(p.w, v, o[4 * q4 + 3]);
+                    }
+                }
+            }
+            __syncthreads();
+        }
+
+        // Partial of this split (window + block) for every row.
+        const int seg = a.nsplit;
+        if (tid < D) {
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) {
+                if (rr < nr) {
+                    const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
+                    a.part_o[((row * H + h) * a.nseg + seg) * D + tid] = o[rr];
+                }
+            }
+        }
+        float* ml_s = alph;  // reuse: (m, l) of each row for the merge
+#pragma unroll
+        for (int i = 0; i < kRows / 4; ++i) {
+            const int rr = warp + 4 * i;
+            if (rr >= nr) break;
+            if (lane == 0) {
+                const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
+                a.part_ml[(row * H + h) * a.nseg + seg] = make_float2(mrow[i], lrow[i]);
+            }
+        }
+        __syncthreads();  // alph no longer read
+#pragma unroll
+        for (int i = 0; i < kRows / 4; ++i) {
+            const int rr = warp + 4 * i;
+            if (rr < nr && lane == 0) {
+                ml_s[2 * rr] = mrow[i];
+                ml_s[2 * rr + 1] = lrow[i];
+            }
+        }
+        __threadfence();
+        __syncthreads();
+        const int ndeep = deep_splits_used(A, a.chunk, a.nsplit);
+        if (tid == 0) {
+            int* cnt = a.cnt + ((int64_t)bi * a.nrowchunks + rc) * H + h;
+            const int old = atomicAdd(cnt, 1);
+            const int last = old == ndeep;
+            if (last) *cnt = 0;
+            flags[0] = last;
+            __threadfence();
+        }
+        __syncthreads();
+        if (flags[0]) {
+            // Last to arrive: merge with the deep partials (read past L1, they come from other CTAs).
+            if (tid < D) {
+#pragma unroll
+                for (int rr = 0; rr < kRows; ++rr) {
+                    if (rr >= nr) break;
+                    const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
+                    const int64_t base = (row * H + h) * a.nseg;
+                    float M = ml_s[2 * rr];
+                    for (int sg = 0; sg < ndeep; ++sg) M = fmaxf(M, __ldcg(a.part_ml + base + sg).x);
+                    const float fo = ex2(ml_s[2 * rr] - M);
+                    float L = ml_s[2 * rr + 1] * fo, acc = o[rr] * fo;
+                    for (int sg = 0; sg < ndeep; ++sg) {
+                        const float2 ml = __ldcg(a.part_ml + base + sg);
+                        const float f = ex2(ml.x - M);
+                        L = fmaf(ml.y, f, L);
+                        acc = fmaf(__ldcg(a.part_o + (base + sg) * D + tid), f, acc);
+                    }
+                    reinterpret_cast<__nv_bfloat16*>(a.O)[(row * H + h) * D + tid] = __float2bfloat16_rn(acc / L);
+                    if (tid == 0 && a.lse) a.lse[row * H + h] = (M + log2f(L)) * 0.69314718055994531f;
+                }
+            }
+        }
+    }
+
+    // Completion: the last CTA of this grid waits for the deep-plane grid it may run
+    // beside (programmatic dependent launch), so that this grid ending implies both ended.
+    __syncthreads();
+    if (tid == 0) {
+        const int n = atomicAdd(a.done, 1);
+        if (n == (int)gridDim.x - 1) {
+            *a.done = 0;
+            grid_dependency_wait();
+        }
+    }
+    grid_launch_dependents();
+}
+
+}  // namespace
+
+bool window_supported(int dtype, int d) { return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128); }
+
+cudaError_t launch_window(const VerifyArgs& a, int nbranch, int keys_ub, bool pdl, cudaStream_t st) {
+    const int64_t grid = (int64_t)nbranch * a.nrowchunks * a.s.H;
+    if (grid == 0) return cudaSuccess;
+    if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    int KT = (keys_ub + 7) / 8 * 8;
+    if (KT > 160) KT = 128;
+    if (KT < 8) KT = 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    static bool attrs_set = false;
+    if (!attrs_set) {
+#define RIPE_WIN_ATTR(D_, NR_)                                                                             \
+        cudaFuncSetAttribute(window_kernel<D_, NR_>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024); \
+        cudaFuncSetAttribute(window_kernel<D_, NR_>, cudaFuncAttributePreferredSharedMemoryCarveout,          \
+                             cudaSharedmemCarveoutMaxShared);
+        RIPE_WIN_ATTR(64, 4) RIPE_WIN_ATTR(64, 8) RIPE_WIN_ATTR(64, 16)
+        RIPE_WIN_ATTR(96, 4) RIPE_WIN_ATTR(96, 8) RIPE_WIN_ATTR(96, 16)
+        RIPE_WIN_ATTR(128, 4) RIPE_WIN_ATTR(128, 8) RIPE_WIN_ATTR(128, 16)
+#undef RIPE_WIN_ATTR
+        attrs_set = true;
+    }
+    const int rows = a.ba.max_ntok < kRowChunk ? a.ba.max_ntok : kRowChunk;
+    const int NR = rows <= 4 ? 4 : rows <= 8 ? 8 : 16;
+    cudaError_t e = cudaErrorInvalidValue;
+#define RIPE_WIN_GO(D_, NR_)                                       \
+    if (a.s.d == D_ && NR == NR_) {                                \
+        cfg.dynamicSmemBytes = WinLayout<D_, NR_>::bytes(KT);      \
+        e = cudaLaunchKernelEx(&cfg, window_kernel<D_, NR_>, a, KT); \
+    }
+    RIPE_WIN_GO(64, 4) RIPE_WIN_GO(64, 8) RIPE_WIN_GO(64, 16)
+    RIPE_WIN_GO(96, 4) RIPE_WIN_GO(96, 8) RIPE_WIN_GO(96, 16)
+    RIPE_WIN_GO(128, 4) RIPE_WIN_GO(128, 8) RIPE_WIN_GO(128, 16)
+#undef RIPE_WIN_GO
+    ripe_count_launch();
+    return e;
+}
