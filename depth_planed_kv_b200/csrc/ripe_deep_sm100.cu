@@ -350,12 +350,21 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                     tmem_ld32(lane_addr + Lay::S_COL(mt, sb), sc);
                     tmem_ld32(lane_addr + Lay::S_COL(mt, sb) + 32, sc + 32);
                     tmem_wait_ld();
-                    float mx = -INFINITY;
+                    if (nvalid < kN) {
 #pragma unroll
-                    for (int c = 0; c < kN; ++c) {
-                        sc[c] = c < nvalid ? sc[c] * c2 : -INFINITY;
-                        mx = fmaxf(mx, sc[c]);
+                        for (int c = 0; c < kN; ++c)
+                            if (c >= nvalid) sc[c] = -INFINITY;
                     }
+                    // Row max of the raw scores (scale > 0 commutes with max), four chains.
+                    float m4[4] = {sc[0], sc[1], sc[2], sc[3]};
+#pragma unroll
+                    for (int c = 4; c < kN; c += 4) {
+                        m4[0] = fmaxf(m4[0], sc[c]);
+                        m4[1] = fmaxf(m4[1], sc[c + 1]);
+                        m4[2] = fmaxf(m4[2], sc[c + 2]);
+                        m4[3] = fmaxf(m4[3], sc[c + 3]);
+                    }
+                    const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
                     // The running max moves only when it grows by more than 2^8 (probabilities
                     // then stay below 256); the O rescale is warp-collective.
                     float alpha = 1.f;
@@ -383,7 +392,9 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                         }
                         tmem_wait_st();
                     }
-                    float sum = 0.f;
+                    // p = 2^(s*scale*log2e - m): one FMA and one ex2 per score.
+                    const float nm = -m[mt];
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f};
                     uint8_t* prow = sP + (sb * MT + mt) * Lay::P_BUF + t * 64;
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
@@ -392,9 +403,9 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                             uint32_t w[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const float x0 = ex2(sc[c * 32 + gq * 8 + 2 * e] - m[mt]);
-                                const float x1 = ex2(sc[c * 32 + gq * 8 + 2 * e + 1] - m[mt]);
-                                sum += x0 + x1;
+                                const float x0 = ex2(fmaf(sc[c * 32 + gq * 8 + 2 * e], c2, nm));
+                                const float x1 = ex2(fmaf(sc[c * 32 + gq * 8 + 2 * e + 1], c2, nm));
+                                s4[e] += x0 + x1;
                                 __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
                                 w[e] = *reinterpret_cast<uint32_t*>(&b2);
                             }
@@ -402,7 +413,7 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                                 make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }
-                    l[mt] = l[mt] * alpha + sum;
+                    l[mt] = l[mt] * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
                 }
                 if (!ok) break;
                 fence_proxy_async_smem();
@@ -428,7 +439,6 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                                 dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
                         }
                     }
-                    __threadfence();
                     tc_fence_before();
                 }
             }
@@ -445,6 +455,7 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     if (total_it > 0 && !*abort_flag) {
         const int ndeep = deep_splits_used(G.A, a.chunk, a.nsplit);
         if (warp == 0) {
+            __threadfence();  // releases the partials written before the barrier above
             for (int i = lane; i < G.nb; i += 32) {
                 int mask = 0;
                 const int nrc = (bt[i].ntok + kWinRows - 1) / kWinRows;
@@ -466,6 +477,8 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             const int row = group_row(bt, G.nb, rl, &bi, &j);
             if (row < 0 || !((bt[bi].last_mask >> (j / kWinRows)) & 1)) continue;
             const int64_t base = ((int64_t)row * s.H + h) * nseg;
+            // Deep splits in order, then the window partial -- the same operation order as
+            // the window-side merge, so the result does not depend on who merges.
             float mls[2 * 9];
             const int np = ndeep < 8 ? ndeep : 8;
             float M = -INFINITY;
@@ -473,14 +486,14 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 const float2 ml = __ldcg(a.part_ml + base + (sg < np ? sg : a.nsplit));
                 mls[2 * sg] = ml.x;
                 mls[2 * sg + 1] = ml.y;
-                M = fmaxf(M, ml.x);
             }
+            for (int sg = 0; sg < np; ++sg) M = fmaxf(M, mls[2 * sg]);
+            M = fmaxf(M, mls[2 * np]);
             float L = 0.f;
             for (int sg = 0; sg <= np; ++sg) {
                 mls[2 * sg] = ex2(mls[2 * sg] - M);
                 L = fmaf(mls[2 * sg + 1], mls[2 * sg], L);
             }
-            const float inv = 1.f / L;
             __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ((int64_t)row * s.H + h) * D;
 #pragma unroll 2
             for (int c = 0; c < D; c += 8) {
@@ -500,7 +513,7 @@ deep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 uint32_t w4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * e] / L, acc[2 * e + 1] / L);
                     w4[e] = *reinterpret_cast<uint32_t*>(&b2);
                 }
                 *reinterpret_cast<uint4*>(orow + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);

@@ -92,18 +92,6 @@ __global__ void __launch_bounds__(kThreads) window_kernel(VerifyArgs a, int KT) 
         const int slot0 = A % s.Wcap;  // ring slot of the first window position
         const int64_t ring_base = ring ? ring_row(s, a.layer, b, h, r, 0) : 0;
         if (tid == 0) flags[1] = 0;
-        for (int e = tid; e < kRows * D; e += kThreads) {
-            const int rr = e / D, c = e % D;
-            float qv = 0.f;
-            if (rr < nr) {
-                const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
-                qv = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.Q)[(row * H + h) * D + c]) *
-                     a.scale_log2;
-            }
-            q_s[rr * D + c] = qv;
-        }
-        __syncthreads();
-
         float mrow[kRows / 4], lrow[kRows / 4];  // warp w: rows w, w+4, w+8, w+12
 #pragma unroll
         for (int i = 0; i < kRows / 4; ++i) { mrow[i] = -INFINITY; lrow[i] = 0.f; }
@@ -141,6 +129,31 @@ __global__ void __launch_bounds__(kThreads) window_kernel(VerifyArgs a, int KT) 
                 cp_async16(sV + (size_t)kk * ROWB + 16 * v, vs + 16 * v);
             }
             cp_async_commit();
+            if (t == 0) {
+                // q rows (pre-scaled to log2 units) while the first tile is in flight;
+                // rows past nr are zero so every row loop can run all NR rows.
+                constexpr int QV = D / 8;  // 16-byte vectors per q row
+                for (int e = tid; e < kRows * QV; e += kThreads) {
+                    const int rr = e / QV, v = e - rr * QV;
+                    uint4 x = make_uint4(0, 0, 0, 0);
+                    if (rr < nr) {
+                        const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
+                        x = *reinterpret_cast<const uint4*>(a.Q + (row * H + h) * ROWB + 16 * v);
+                    }
+                    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                    float4 lo, hi;
+                    lo.x = __uint_as_float(xw[0] << 16) * a.scale_log2;
+                    lo.y = __uint_as_float(xw[0] & 0xFFFF0000u) * a.scale_log2;
+                    lo.z = __uint_as_float(xw[1] << 16) * a.scale_log2;
+                    lo.w = __uint_as_float(xw[1] & 0xFFFF0000u) * a.scale_log2;
+                    hi.x = __uint_as_float(xw[2] << 16) * a.scale_log2;
+                    hi.y = __uint_as_float(xw[2] & 0xFFFF0000u) * a.scale_log2;
+                    hi.z = __uint_as_float(xw[3] << 16) * a.scale_log2;
+                    hi.w = __uint_as_float(xw[3] & 0xFFFF0000u) * a.scale_log2;
+                    *reinterpret_cast<float4*>(q_s + rr * D + 8 * v) = lo;
+                    *reinterpret_cast<float4*>(q_s + rr * D + 8 * v + 4) = hi;
+                }
+            }
             cp_async_wait_all();
             __syncthreads();
             // A. scores in log2 units: thread = key; q rows broadcast from shared memory
@@ -259,11 +272,11 @@ __global__ void __launch_bounds__(kThreads) window_kernel(VerifyArgs a, int KT) 
                 ml_s[2 * rr + 1] = lrow[i];
             }
         }
-        __threadfence();
         __syncthreads();
         const int ndeep = deep_splits_used(A, a.chunk, a.nsplit);
         if (tid == 0) {
             int* cnt = a.cnt + ((int64_t)bi * a.nrowchunks + rc) * H + h;
+            __threadfence();  // releases every thread's partial (ordered before by the barrier)
             const int old = atomicAdd(cnt, 1);
             const int last = old == ndeep;
             if (last) *cnt = 0;
@@ -272,23 +285,49 @@ __global__ void __launch_bounds__(kThreads) window_kernel(VerifyArgs a, int KT) 
         }
         __syncthreads();
         if (flags[0]) {
-            // Last to arrive: merge with the deep partials (read past L1, they come from other CTAs).
+            // Last to arrive: merge with the deep partials (read past L1, they come from
+            // other CTAs).  Row by row, all of a row's loads are issued before use.
+            constexpr int MAXS = 8;
             if (tid < D) {
-#pragma unroll
-                for (int rr = 0; rr < kRows; ++rr) {
-                    if (rr >= nr) break;
+#pragma unroll 1
+                for (int rr = 0; rr < nr; ++rr) {
                     const int64_t row = br.row0 + (int64_t)(j0 + rr) * br.stride;
                     const int64_t base = (row * H + h) * a.nseg;
-                    float M = ml_s[2 * rr];
-                    for (int sg = 0; sg < ndeep; ++sg) M = fmaxf(M, __ldcg(a.part_ml + base + sg).x);
-                    const float fo = ex2(ml_s[2 * rr] - M);
-                    float L = ml_s[2 * rr + 1] * fo, acc = o[rr] * fo;
-                    for (int sg = 0; sg < ndeep; ++sg) {
-                        const float2 ml = __ldcg(a.part_ml + base + sg);
-                        const float f = ex2(ml.x - M);
-                        L = fmaf(ml.y, f, L);
-                        acc = fmaf(__ldcg(a.part_o + (base + sg) * D + tid), f, acc);
+                    float mv[MAXS], lv[MAXS], ov[MAXS];
+#pragma unroll
+                    for (int sg = 0; sg < MAXS; ++sg) {
+                        mv[sg] = -INFINITY;
+                        lv[sg] = 0.f;
+                        ov[sg] = 0.f;
+                        if (sg < ndeep) {
+                            const float2 ml = __ldcg(a.part_ml + base + sg);
+                            mv[sg] = ml.x;
+                            lv[sg] = ml.y;
+                            ov[sg] = __ldcg(a.part_o + (base + sg) * D + tid);
+                        }
                     }
+                    float orow = 0.f;
+#pragma unroll
+                    for (int q = 0; q < kRows; ++q)
+                        if (q == rr) orow = o[q];
+                    // Same operation order as the deep-side merge (deep splits in order,
+                    // then the window partial), so the result does not depend on who merges.
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int sg = 0; sg < MAXS; ++sg) M = fmaxf(M, mv[sg]);
+                    M = fmaxf(M, ml_s[2 * rr]);
+                    float L = 0.f, acc = 0.f;
+#pragma unroll
+                    for (int sg = 0; sg < MAXS; ++sg) {
+                        if (sg < ndeep) {
+                            const float f = ex2(mv[sg] - M);
+                            L = fmaf(lv[sg], f, L);
+                            acc = fmaf(ov[sg], f, acc);
+                        }
+                    }
+                    const float fo = ex2(ml_s[2 * rr] - M);
+                    L = fmaf(ml_s[2 * rr + 1], fo, L);
+                    acc = fmaf(orow, fo, acc);
                     reinterpret_cast<__nv_bfloat16*>(a.O)[(row * H + h) * D + tid] = __float2bfloat16_rn(acc / L);
                     if (tid == 0 && a.lse) a.lse[row * H + h] = (M + log2f(L)) * 0.69314718055994531f;
                 }
