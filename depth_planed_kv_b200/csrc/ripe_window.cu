@@ -348,9 +348,372 @@ __global__ void __launch_bounds__(kThreads) window_kernel(VerifyArgs a, int KT) 
     grid_launch_dependents();
 }
 
+// ---------------------------------------------------------------------------
+// Grouped variant: G units (consecutive branches -- for all-depths calls,
+// consecutive loop depths -- of one head and row chunk) per CTA of 256 threads,
+// so every phase has work for all threads and the barriers, copies, counters and
+// merges are shared by G units.  Used when every unit's keys fit one tile.
+// ---------------------------------------------------------------------------
+
+template <int D, int NR, int G>
+struct GroupLayout {
+    static constexpr int ROWB = D * 2;
+    static constexpr int KSTR = ROWB + 16;
+    static constexpr int NVEC = ROWB / 16;
+    // per unit: K (padded), V, q (fp32), scores [row][key], probabilities [key][row]
+    __host__ __device__ static size_t unit_bytes(int KTU) {
+        return (size_t)KTU * (KSTR + ROWB) + (size_t)NR * D * 4 + (size_t)2 * NR * KTU * 4;
+    }
+    __host__ __device__ static size_t bytes(int KTU) { return 512 + G * unit_bytes(KTU) + G * NR * 8; }
+};
+
+struct UnitInfo {
+    const char *kring, *vring;  // plane r ring base (r < R) or deep plane base (r == R)
+    int nk, nwin, nr, j0, row0, stride, bi, rc, h, A, slot0, ring, ndeep, last;
+};
+
+template <int D, int NR, int G>
+__global__ void __launch_bounds__(64 * G) wgroup_kernel(VerifyArgs a, int KTU) {
+    constexpr int kGThreads = 64 * G;  // two warps per unit
+    using namespace sm100;
+    using Lay = GroupLayout<D, NR, G>;
+    constexpr int ROWB = Lay::ROWB, KSTR = Lay::KSTR, NVEC = Lay::NVEC;
+    constexpr int NCP = D / 2;  // channel pairs per unit
+    extern __shared__ __align__(128) uint8_t smem[];
+    UnitInfo* ui = reinterpret_cast<UnitInfo*>(smem);  // G entries (< 512 bytes)
+    uint8_t* ubase = smem + 512;
+    float* mls = reinterpret_cast<float*>(ubase + G * Lay::unit_bytes(KTU));  // [G][NR][2]
+    auto uK = [&](int u) { return ubase + u * Lay::unit_bytes(KTU); };
+    auto uV = [&](int u) { return uK(u) + (size_t)KTU * KSTR; };
+    auto uQ = [&](int u) { return reinterpret_cast<float*>(uV(u) + (size_t)KTU * ROWB); };
+    auto uS = [&](int u) { return uQ(u) + NR * D; };
+    auto uP = [&](int u) { return uS(u) + (size_t)NR * KTU; };
+
+    const StoreView& s = a.s;
+    const int H = s.H;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int ngroups_b = (a.ba.nbranch + G - 1) / G;
+
+    // ---- unit descriptors (one thread per unit)
+    if (tid < G) {
+        int64_t gidx = blockIdx.x;
+        const int gb = (int)(gidx % ngroups_b);
+        gidx /= ngroups_b;
+        const int rc = (int)(gidx % a.nrowchunks);
+        const int h = (int)(gidx / a.nrowchunks);
+        const int bi = gb * G + tid;
+        UnitInfo info{};
+        info.nk = 0;
+        if (bi < a.ba.nbranch) {
+            const Branch br = load_branch(a.ba, s.R, s.Bmax, bi);
+            if (!br.ok && rc == 0 && h == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
+            const int j0 = rc * kRowChunk;
+            if (br.ok && j0 < br.ntok) {
+                const int b = br.seq, r = br.depth;
+                const int T = context_length(s.len, a.ctx, s.err, b, h == 0 && rc == 0);
+                const int A = min(s.ws[b], T);
+                info.nr = min(NR, br.ntok - j0);
+                info.j0 = j0;
+                info.nwin = T - A;
+                info.nk = info.nwin + j0 + info.nr;
+                info.row0 = br.row0;
+                info.stride = br.stride;
+                info.bi = bi;
+                info.rc = rc;
+                info.h = h;
+                info.A = A;
+                info.ring = r < s.R;
+                info.slot0 = A % s.Wcap;
+                info.kring = info.ring ? s.kwin + ring_row(s, a.layer, b, h, r, 0) : s.kdeep + deep_row(s, a.layer, b, h, A);
+                info.vring = info.ring ? s.vwin + ring_row(s, a.layer, b, h, r, 0) : s.vdeep + deep_row(s, a.layer, b, h, A);
+                info.ndeep = deep_splits_used(A, a.chunk, a.nsplit);
+            }
+        }
+        ui[tid] = info;
+    }
+    __syncthreads();
+    int nkmax = 0, total = 0;
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+        nkmax = max(nkmax, ui[u].nk);
+        total += ui[u].nk;
+    }
+
+    if (total > 0) {
+        // ---- copies: one K/V row per thread-iteration (K padded, V dense)
+        for (int pidx = tid; pidx < total; pidx += kGThreads) {
+            int u = 0, key = pidx;
+#pragma unroll
+            for (int q = 0; q < G - 1; ++q)
+                if (u == q && key >= ui[q].nk) { key -= ui[q].nk; u = q + 1; }
+            const UnitInfo& U = ui[u];
+            const char *kp, *vp;
+            if (key < U.nwin) {
+                if (U.ring) {
+                    int slot = U.slot0 + key;
+                    if (slot >= s.Wcap) slot -= s.Wcap;
+                    kp = U.kring + (int64_t)slot * ROWB;
+                    vp = U.vring + (int64_t)slot * ROWB;
+                } else {
+                    kp = U.kring + (int64_t)key * ROWB;
+                    vp = U.vring + (int64_t)key * ROWB;
+                }
+            } else {
+                const int64_t row = U.row0 + (int64_t)(key - U.nwin) * U.stride;
+                kp = a.Kb + (row * H + U.h) * ROWB;
+                vp = a.Vb + (row * H + U.h) * ROWB;
+            }
+            uint8_t* dk = uK(u) + (size_t)key * KSTR;
+            uint8_t* dv = uV(u) + (size_t)key * ROWB;
+#pragma unroll
+            for (int v = 0; v < NVEC; ++v) {
+                cp_async16(dk + 16 * v, kp + 16 * v);
+                cp_async16(dv + 16 * v, vp + 16 * v);
+            }
+        }
+        cp_async_commit();
+        // ---- q rows (log2 units; rows past nr are zero) while the copies fly
+        for (int e = tid; e < G * NR * NVEC; e += kGThreads) {
+            const int u = e / (NR * NVEC), rem = e - u * NR * NVEC;
+            const int rr = rem / NVEC, v = rem - rr * NVEC;
+            const UnitInfo& U = ui[u];
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (U.nk > 0 && rr < U.nr) {
+                const int64_t row = U.row0 + (int64_t)(U.j0 + rr) * U.stride;
+                x = *reinterpret_cast<const uint4*>(a.Q + (row * H + U.h) * ROWB + 16 * v);
+            }
+            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+            float* dst = uQ(u) + rr * D + 8 * v;
+            float4 lo, hi;
+            lo.x = __uint_as_float(xw[0] << 16) * a.scale_log2;
+            lo.y = __uint_as_float(xw[0] & 0xFFFF0000u) * a.scale_log2;
+            lo.z = __uint_as_float(xw[1] << 16) * a.scale_log2;
+            lo.w = __uint_as_float(xw[1] & 0xFFFF0000u) * a.scale_log2;
+            hi.x = __uint_as_float(xw[2] << 16) * a.scale_log2;
+            hi.y = __uint_as_float(xw[2] & 0xFFFF0000u) * a.scale_log2;
+            hi.z = __uint_as_float(xw[3] << 16) * a.scale_log2;
+            hi.w = __uint_as_float(xw[3] & 0xFFFF0000u) * a.scale_log2;
+            *reinterpret_cast<float4*>(dst) = lo;
+            *reinterpret_cast<float4*>(dst + 4) = hi;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+
+        // ---- A. scores: thread = (unit, key); the K row read once for all rows
+        for (int pidx = tid; pidx < total; pidx += kGThreads) {
+            int u = 0, key = pidx;
+#pragma unroll
+            for (int q = 0; q < G - 1; ++q)
+                if (u == q && key >= ui[q].nk) { key -= ui[q].nk; u = q + 1; }
+            const UnitInfo& U = ui[u];
+            const float* qb = uQ(u);
+            const uint4* krow = reinterpret_cast<const uint4*>(uK(u) + (size_t)key * KSTR);
+            float acc[NR];
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr) acc[rr] = 0.f;
+#pragma unroll 4
+            for (int v = 0; v < NVEC; ++v) {
+                const uint4 x = krow[v];
+                const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                float kf[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    kf[2 * e] = __uint_as_float(xw[e] << 16);
+                    kf[2 * e + 1] = __uint_as_float(xw[e] & 0xFFFF0000u);
+                }
+#pragma unroll
+                for (int rr = 0; rr < NR; ++rr) {
+                    const float4 qa = *reinterpret_cast<const float4*>(qb + rr * D + 8 * v);
+                    const float4 qc = *reinterpret_cast<const float4*>(qb + rr * D + 8 * v + 4);
+                    acc[rr] = fmaf(qa.x, kf[0], acc[rr]);
+                    acc[rr] = fmaf(qa.y, kf[1], acc[rr]);
+                    acc[rr] = fmaf(qa.z, kf[2], acc[rr]);
+                    acc[rr] = fmaf(qa.w, kf[3], acc[rr]);
+                    acc[rr] = fmaf(qc.x, kf[4], acc[rr]);
+                    acc[rr] = fmaf(qc.y, kf[5], acc[rr]);
+                    acc[rr] = fmaf(qc.z, kf[6], acc[rr]);
+                    acc[rr] = fmaf(qc.w, kf[7], acc[rr]);
+                }
+            }
+            float* sc = uS(u);
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr) {
+                const bool masked = rr >= U.nr || (key >= U.nwin && key - U.nwin > U.j0 + rr);
+                sc[rr * KTU + key] = masked ? -INFINITY : acc[rr];
+            }
+        }
+        __syncthreads();
+
+        // ---- B. softmax: warp = (unit, row)
+        for (int pr = warp; pr < G * NR; pr += kGThreads / 32) {
+            const int u = pr / NR, rr = pr - u * NR;
+            const UnitInfo& U = ui[u];
+            const int nk = U.nk;
+            const float* srow = uS(u) + rr * KTU;
+            float* pt = uP(u);
+            float mt = -INFINITY;
+            for (int kk = lane; kk < nk; kk += 32) mt = fmaxf(mt, srow[kk]);
+            mt = warp_max(mt);
+            float sum = 0.f;
+            for (int kk = lane; kk < nk; kk += 32) {
+                const float p = mt == -INFINITY ? 0.f : ex2(srow[kk] - mt);
+                pt[kk * NR + rr] = p;
+                sum += p;
+            }
+            sum = warp_sum(sum);
+            if (lane == 0) {
+                mls[(u * NR + rr) * 2] = mt;
+                mls[(u * NR + rr) * 2 + 1] = sum;
+            }
+        }
+        __syncthreads();
+
+        // ---- C. o = P V: thread = (unit, channel pair)
+        for (int pc = tid; pc < G * NCP; pc += kGThreads) {
+            const int u = pc / NCP, cp2 = pc - u * NCP;
+            const UnitInfo& U = ui[u];
+            if (U.nk == 0) continue;
+            const uint32_t* vcol = reinterpret_cast<const uint32_t*>(uV(u)) + cp2;
+            const float4* pk = reinterpret_cast<const float4*>(uP(u));
+            float o0[NR], o1[NR];
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr) { o0[rr] = 0.f; o1[rr] = 0.f; }
+#pragma unroll 4
+            for (int kk = 0; kk < U.nk; ++kk) {
+                const uint32_t w2 = vcol[kk * (ROWB / 4)];
+                const float v0 = __uint_as_float(w2 << 16), v1 = __uint_as_float(w2 & 0xFFFF0000u);
+#pragma unroll
+                for (int q4 = 0; q4 < NR / 4; ++q4) {
+                    const float4 p = pk[kk * (NR / 4) + q4];
+                    o0[4 * q4] = fmaf(p.x, v0, o0[4 * q4]);         o1[4 * q4] = fmaf(p.x, v1, o1[4 * q4]);
+                    o0[4 * q4 + 1] = fmaf(p.y, v0, o0[4 * q4 + 1]); o1[4 * q4 + 1] = fmaf(p.y, v1, o1[4 * q4 + 1]);
+                    o0[4 * q4 + 2] = fmaf(p.z, v0, o0[4 * q4 + 2]); o1[4 * q4 + 2] = fmaf(p.z, v1, o1[4 * q4 + 2]);
+                    o0[4 * q4 + 3] = fmaf(p.w, v0, o0[4 * q4 + 3]); o1[4 * q4 + 3] = fmaf(p.w, v1, o1[4 * q4 + 3]);
+                }
+            }
+            // partial of this split (window + block)
+            const int seg = a.nsplit;
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr) {
+                if (rr < U.nr) {
+                    const int64_t row = U.row0 + (int64_t)(U.j0 + rr) * U.stride;
+                    const int64_t pi = (row * H + U.h) * a.nseg + seg;
+                    *reinterpret_cast<float2*>(a.part_o + pi * D + 2 * cp2) = make_float2(o0[rr], o1[rr]);
+                    if (cp2 == 0) a.part_ml[pi] = make_float2(mls[(u * NR + rr) * 2], mls[(u * NR + rr) * 2 + 1]);
+                }
+            }
+            // keep o for a possible merge: stash it in the (now free) K tile
+            float* stash = reinterpret_cast<float*>(uK(u));
+#pragma unroll
+            for (int rr = 0; rr < NR; ++rr) {
+                stash[rr * D + 2 * cp2] = o0[rr];
+                stash[rr * D + 2 * cp2 + 1] = o1[rr];
+            }
+        }
+        __syncthreads();
+
+        // ---- arrivals: one thread per unit
+        if (tid < G) {
+            UnitInfo& U = ui[tid];
+            if (U.nk > 0) {
+                int* cnt = a.cnt + ((int64_t)U.bi * a.nrowchunks + U.rc) * H + U.h;
+                __threadfence();  // releases the CTA's partials (ordered before by the barrier)
+                U.last = atomicAdd(cnt, 1) == U.ndeep;
+                if (U.last) *cnt = 0;
+                __threadfence();
+            } else {
+                U.last = 0;
+            }
+        }
+        __syncthreads();
+
+        // ---- merge where this CTA arrived last: thread = (unit, channel pair);
+        // deep splits in order, then the window partial (same order as the deep side).
+        for (int pc = tid; pc < G * NCP; pc += kGThreads) {
+            const int u = pc / NCP, cp2 = pc - u * NCP;
+            const UnitInfo& U = ui[u];
+            if (U.nk == 0 || !U.last) continue;
+            const float* stash = reinterpret_cast<const float*>(uK(u));
+            for (int rr = 0; rr < U.nr; ++rr) {
+                const int64_t row = U.row0 + (int64_t)(U.j0 + rr) * U.stride;
+                const int64_t base = (row * H + U.h) * a.nseg;
+                const float mw = mls[(u * NR + rr) * 2], lw = mls[(u * NR + rr) * 2 + 1];
+                float M = mw;
+                for (int sg = 0; sg < U.ndeep; ++sg) M = fmaxf(M, __ldcg(a.part_ml + base + sg).x);
+                float L = 0.f, acc0 = 0.f, acc1 = 0.f;
+                for (int s0 = 0; s0 < U.ndeep; s0 += 4) {
+                    float mv[4], lv[4];
+                    float2 ov[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (s0 + q < U.ndeep) {
+                            const float2 ml = __ldcg(a.part_ml + base + s0 + q);
+                            mv[q] = ml.x;
+                            lv[q] = ml.y;
+                            ov[q] = __ldcg(reinterpret_cast<const float2*>(a.part_o + (base + s0 + q) * D) + cp2);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (s0 + q < U.ndeep) {
+                            const float f = ex2(mv[q] - M);
+                            L = fmaf(lv[q], f, L);
+                            acc0 = fmaf(ov[q].x, f, acc0);
+                            acc1 = fmaf(ov[q].y, f, acc1);
+                        }
+                    }
+                }
+                const float fo = ex2(mw - M);
+                L = fmaf(lw, fo, L);
+                acc0 = fmaf(stash[rr * D + 2 * cp2], fo, acc0);
+                acc1 = fmaf(stash[rr * D + 2 * cp2 + 1], fo, acc1);
+                *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(a.O) + (row * H + U.h) * D +
+                                                   2 * cp2) = __floats2bfloat162_rn(acc0 / L, acc1 / L);
+                if (cp2 == 0 && a.lse) a.lse[row * H + U.h] = (M + log2f(L)) * 0.69314718055994531f;
+            }
+        }
+    }
+    (void)nkmax;
+
+    // Completion: the last CTA of this grid waits for the deep-plane grid it may run beside.
+    __syncthreads();
+    if (tid == 0) {
+        const int n = atomicAdd(a.done, 1);
+        if (n == (int)gridDim.x - 1) {
+            *a.done = 0;
+            grid_dependency_wait();
+        }
+    }
+    grid_launch_dependents();
+}
+
 }  // namespace
 
 bool window_supported(int dtype, int d) { return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128); }
+
+template <int D, int NR, int G>
+cudaError_t launch_group_t(cudaLaunchConfig_t cfg, const VerifyArgs& a, int KTU) {
+    static bool set = false;
+    if (!set) {
+        cudaFuncSetAttribute(wgroup_kernel<D, NR, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaFuncSetAttribute(wgroup_kernel<D, NR, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+        set = true;
+    }
+    const int64_t groups = (int64_t)(a.ba.nbranch + G - 1) / G * a.nrowchunks * a.s.H;
+    if (groups > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3((unsigned)groups);
+    cfg.blockDim = dim3(64 * G);
+    cfg.dynamicSmemBytes = GroupLayout<D, NR, G>::bytes(KTU);
+    return cudaLaunchKernelEx(&cfg, wgroup_kernel<D, NR, G>, a, KTU);
+}
+
+template <int D, int NR>
+cudaError_t launch_group_d(cudaLaunchConfig_t cfg, const VerifyArgs& a, int KTU, int G) {
+    if (G == 4) return launch_group_t<D, NR, 4>(cfg, a, KTU);
+    if (G == 2) return launch_group_t<D, NR, 2>(cfg, a, KTU);
+    return launch_group_t<D, NR, 1>(cfg, a, KTU);
+}
 
 cudaError_t launch_window(const VerifyArgs& a, int nbranch, int keys_ub, bool pdl, cudaStream_t st) {
     const int64_t grid = (int64_t)nbranch * a.nrowchunks * a.s.H;
@@ -368,6 +731,31 @@ cudaError_t launch_window(const VerifyArgs& a, int nbranch, int keys_ub, bool pd
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
+    const int rows = a.ba.max_ntok < kRowChunk ? a.ba.max_ntok : kRowChunk;
+    const int NR = rows <= 4 ? 4 : rows <= 8 ? 8 : 16;
+
+    // Grouped kernel when every unit's keys fit one tile and NR <= 8: as many units
+    // per CTA as keep the CTA within ~70 KB of shared memory (three per SM).
+    if (keys_ub <= 160 && NR <= 8) {
+        int KTU = (keys_ub + 7) / 8 * 8;
+        const int min_ktu = (NR * a.s.d * 4 + (2 * a.s.d + 16) - 1) / (2 * a.s.d + 16);  // o stash fits the K tile
+        if (KTU < min_ktu) KTU = (min_ktu + 7) / 8 * 8;
+        const size_t unit = (size_t)KTU * (4 * a.s.d + 16) + (size_t)NR * a.s.d * 4 + (size_t)2 * NR * KTU * 4;
+        int G = 4;
+        while (G > 1 && 512 + G * unit + G * NR * 8 > 72 * 1024) G /= 2;
+        cudaError_t e = cudaErrorInvalidValue;
+        switch (a.s.d * 16 + NR) {
+            case 64 * 16 + 4: e = launch_group_d<64, 4>(cfg, a, KTU, G); break;
+            case 64 * 16 + 8: e = launch_group_d<64, 8>(cfg, a, KTU, G); break;
+            case 96 * 16 + 4: e = launch_group_d<96, 4>(cfg, a, KTU, G); break;
+            case 96 * 16 + 8: e = launch_group_d<96, 8>(cfg, a, KTU, G); break;
+            case 128 * 16 + 4: e = launch_group_d<128, 4>(cfg, a, KTU, G); break;
+            case 128 * 16 + 8: e = launch_group_d<128, 8>(cfg, a, KTU, G); break;
+        }
+        ripe_count_launch();
+        return e;
+    }
+
     static bool attrs_set = false;
     if (!attrs_set) {
 #define RIPE_WIN_ATTR(D_, NR_)                                                                             \
@@ -380,8 +768,6 @@ cudaError_t launch_window(const VerifyArgs& a, int nbranch, int keys_ub, bool pd
 #undef RIPE_WIN_ATTR
         attrs_set = true;
     }
-    const int rows = a.ba.max_ntok < kRowChunk ? a.ba.max_ntok : kRowChunk;
-    const int NR = rows <= 4 ? 4 : rows <= 8 ? 8 : 16;
     cudaError_t e = cudaErrorInvalidValue;
 #define RIPE_WIN_GO(D_, NR_)                                       \
     if (a.s.d == D_ && NR == NR_) {                                \
