@@ -104,12 +104,6 @@ int ensure_workspace(ripe_cache_s* c, size_t need, cudaStream_t st) {
         cudaGetLastError();
         return fail(RIPE_ERR_OOM, "cudaMalloc(%zu) for verify scratch failed", sz);
     }
-    // Fresh scratch: the arrival counters at its start must read zero.
-    cudaError_t e = cudaMemset(p, 0, sz < ((size_t)1 << 20) ? sz : ((size_t)1 << 20));
-    if (e != cudaSuccess) {
-        cudaFree(p);
-        return cuda_fail(e, "zeroing the verify scratch");
-    }
     c->work = p;
     c->work_bytes = sz;
     return RIPE_OK;
@@ -127,9 +121,6 @@ int verify_common(ripe_cache_s* c, int layer, const BranchArgs& ba, const void* 
     if (!(scale == scale) || isinf(scale)) return fail(RIPE_ERR_INVALID_ARG, "scale is not finite");
     if (scale == 0.f) scale = 1.0f / sqrtf((float)c->d);
     const VerifyPlan plan = plan_verify(c, ba.nbranch, ba.nrows, ba.max_ntok, ba.table == nullptr);
-    if (plan.counters > verify_max_counters())
-        return fail(RIPE_ERR_CAPACITY, "%lld (branch, row chunk, head) units in one call; at most %lld",
-                    (long long)plan.counters, (long long)verify_max_counters());
     int rc = ensure_workspace(c, plan.work_bytes, st);
     if (rc != RIPE_OK) return rc;
     cudaError_t e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, c->work, st);
@@ -212,7 +203,7 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
     c->kwin = c->base + y.kwin; c->vwin = c->base + y.vwin;
     c->len = (int32_t*)(c->base + y.len); c->ws = (int32_t*)(c->base + y.ws);
     c->err = (int32_t*)(c->base + y.err);
-    c->tc_ready = deep_tc_supported(dtype, d) && make_deep_tensor_maps(c) == 0;
+    c->tc_ready = fused_supported(dtype, d) && make_deep_tensor_maps(c) == 0;
     // Zeroed store: key tiles that overrun a region read finite values.
     cudaError_t e = cudaMemset(c->base, 0, y.total);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -381,12 +372,6 @@ int ripe_get_device_error(ripe_cache_t c, int32_t* code_host, ripe_stream_t stre
     cudaError_t e = cudaMemcpyAsync(code_host, c->err, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(c->err, 0, sizeof(int32_t), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    // A kernel that gave up part-way may have left arrival counters set: clear them.
-    if (e == cudaSuccess && *code_host != 0) {
-        e = reset_verify_counters(c->work, st);
-        if (e == cudaSuccess) e = reset_noalloc_counters(st);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    }
     return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "get_device_error");
 }
 

@@ -1,0 +1,988 @@
+// ripe_fused_sm100.cu -- RIPE verify-attention of one layer in one sm_100a kernel.
+//
+// Every query row of a sequence -- all draft tokens at all loop depths, and every
+// LoopSpec branch -- reads the same deepest plane R outside the window, while a
+// row at depth r reads plane r of the positions still inside the window and the
+// draft-block tokens of its own branch (RIPE abstract, sentence introducing RIPE;
+// LoopSpec article on mixed-depth branches in one batched call).
+//
+// One CTA serves one (sequence group, head, split of the deep region):
+//
+//   deep region (warps 0-5): the group's rows are stacked into 128-row tiles and
+//     S = Q K^T (tcgen05.mma, fp32 in TMEM) -> online softmax on CUDA cores ->
+//     O += P V (tcgen05.mma, fp32 in TMEM)
+//   runs over this split's chunk of plane R, K and V streamed by TMA through a
+//   ring of shared-memory stages.  Warps 0-3 own TMEM lanes 0-127 (one row each)
+//   and do Q staging, softmax and the epilogue; warp 4 lane 0 issues TMA; warp 5
+//   allocates TMEM and its lane 0 issues the MMAs.
+//
+//   window planes and draft block (warps 6..6+NW-1): the keys differ from depth
+//   to depth, so nothing stacks across depths; a unit is one branch's chunk of
+//   <= 8 rows.  Each window warp streams its units' keys 16 at a time through its
+//   own ring of cp.async stages and runs both products on warp-level MMA tiles
+//   (m16n8k16) in the transposed form S^T = K Q^T, O^T = V^T P^T: keys and
+//   channels fill the 16-row side and the <= 8 query rows the 8-column side, and
+//   P^T reaches the B operand by an 8x8 transpose (movmatrix).
+//
+// The splits of one (group, head) form a thread-block cluster.  Each CTA writes
+// its partial results (m in log2 units, l, unnormalised o) to scratch; after a
+// cluster barrier every CTA merges a share of the rows -- deep splits in order,
+// then the window partial: M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L --
+// and writes O and the LSE.  One merger per row, fixed order: bit-reproducible.
+//
+// Shared-memory operand layouts of the deep part (64-byte swizzle, 8-row /
+// 512-byte atoms): Q, K K-major in 32-element column chunks of [rows][64 B];
+// V MN-major (the same chunks read with head-dim as N); P K-major [128][32 keys]
+// chunks written by the softmax threads.  Window stages hold [16 K rows][16 V
+// rows][8 Q rows] at a padded stride of 2*d+16 bytes (conflict-free ldmatrix).
+#include <cuda.h>
+
+#include "ripe_launch.h"
+#include "ripe_verify.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+constexpr int kN = 64;             // deep keys per tile
+constexpr int kDeepThreads = 192;  // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr int kMaxGroupBranches = 64;
+constexpr int kWinRows = 8;   // rows per window unit (the N of an m16n8k16 tile)
+constexpr int kWinKeys = 16;  // keys per window tile (the M of an m16n8k16 tile)
+
+// One branch of the group: its rows, its offset among the group's rows, its
+// depth and the index of its first window unit.
+struct BranchEnt {
+    int row0, stride, ntok, off, depth, uoff;
+};
+
+struct GroupInfo {
+    int first, nb, seq, nrows, T, A, key_begin, key_end, units;
+};
+
+template <int D, int MT, int ST, int NW, int NS>
+struct FusedLayout {
+    static constexpr int NCH = D / 32;               // 64-byte column chunks of the head dim
+    static constexpr int Q_BYTES = MT * NCH * 8192;  // 128 rows x 64 B per chunk
+    static constexpr int KV_STAGE = NCH * 4096;      // 64 keys x 64 B per chunk
+    static constexpr int P_BUF = 2 * 8192;           // one M tile: 2 chunks of 32 keys
+    static constexpr int WSTR = 2 * D + 16;          // window row stride (bytes)
+    static constexpr int WSTAGE = (2 * kWinKeys + kWinRows) * WSTR;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
+    static constexpr int OFF_P = OFF_V + ST * KV_STAGE;
+    static constexpr int OFF_W = OFF_P + 2 * MT * P_BUF;
+    static constexpr int OFF_BAR = OFF_W + NW * NS * WSTAGE;
+    // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int NBAR = 1 + 3 * ST + 7;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_BT = OFF_MISC + 64;
+    static constexpr int BYTES = OFF_BT + kMaxGroupBranches * (int)sizeof(BranchEnt);
+    static constexpr int SMEM = BYTES + 1024;  // alignment slack
+    static constexpr int THREADS = kDeepThreads + 32 * NW;
+    static constexpr uint32_t TMEM_COLS = MT == 1 ? 256 : 512;
+    static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
+    static constexpr uint32_t O_COL(int mt) { return (uint32_t)(MT * 2 * kN + mt * 128); }
+};
+
+// Warp-uniform bounded wait: every lane waits, and all lanes agree on the outcome
+// (the tcgen05.ld/st that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* err) {
+    const bool ok = sm100::mbar_wait(bar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Row (of Q/O) of the group's rl-th query, branches in table order; -1 past the end.
+__device__ int group_row(const BranchEnt* bt, int nb, int rl) {
+    for (int i = 0; i < nb; ++i)
+        if (rl < bt[i].off + bt[i].ntok) return bt[i].row0 + (rl - bt[i].off) * bt[i].stride;
+    return -1;
+}
+
+// Start of the g-th run of equal sequence ids in the branch table (warp-wide).
+__device__ int group_start(const ripe_branch_t* tb, int nbranch, int g, int lane) {
+    int count = 0;
+    for (int base = 0; base < nbranch; base += 32) {
+        const int i = base + lane;
+        const bool st = i < nbranch && (i == 0 || tb[i].seq != tb[i - 1].seq);
+        unsigned m = __ballot_sync(0xffffffffu, st);
+        const int c = __popc(m);
+        if (count + c > g) {
+            for (int k = g - count; k > 0; --k) m &= m - 1;
+            return base + __ffs(m) - 1;
+        }
+        count += c;
+    }
+    return nbranch;
+}
+
+// Window keys of a group: the positions [A, T) still inside the window.  At depth
+// r < R they sit in ring plane r at slots (A .. T-1) mod Wcap; the unit reads the
+// ring in slot order, slots lo .. lo+wk-1 (one contiguous run; slots outside the
+// window are masked and zero-filled, which costs no traffic).  At depth R they
+// are rows A .. T-1 of the deep plane.
+struct WinKeys {
+    int nwin, slot0, lo_ring, wk_ring;
+};
+
+__device__ __forceinline__ WinKeys win_keys(int A, int T, int Wcap) {
+    WinKeys k;
+    k.nwin = T - A;
+    k.slot0 = A % Wcap;
+    if (k.nwin == 0) {
+        k.lo_ring = 0;
+        k.wk_ring = 0;
+    } else if (k.slot0 + k.nwin <= Wcap) {
+        k.lo_ring = k.slot0 & ~15;
+        k.wk_ring = k.slot0 + k.nwin - k.lo_ring;
+    } else {
+        k.lo_ring = 0;
+        k.wk_ring = Wcap;
+    }
+    return k;
+}
+
+// A window unit: rows j0..j0+nr-1 of one branch against nk keys -- wk window keys
+// (ring slots lo.. or deep rows A..), then block tokens 0..j0+nr-1 -- in ntiles
+// tiles of 16 keys.
+struct WinUnit {
+    int row0, stride, depth, j0, nr, wk, lo, nk, ntiles;
+};
+
+// Unit u of the group (warp-collective): its branch is the last one whose first
+// unit is <= u (branches without units share the next branch's first unit).
+__device__ __forceinline__ WinUnit win_unit(const BranchEnt* bt, int nb, int u, const WinKeys& wkeys, int R,
+                                           int lane) {
+    const bool p0 = lane < nb && bt[lane].uoff <= u;
+    const bool p1 = lane + 32 < nb && bt[lane + 32].uoff <= u;
+    const int i = __popc(__ballot_sync(0xffffffffu, p0)) + __popc(__ballot_sync(0xffffffffu, p1)) - 1;
+    const BranchEnt e = bt[i];
+    WinUnit w;
+    w.row0 = e.row0;
+    w.stride = e.stride;
+    w.depth = e.depth;
+    w.j0 = (u - e.uoff) * kWinRows;
+    w.nr = min(kWinRows, e.ntok - w.j0);
+    const bool ring = e.depth < R;
+    w.wk = ring ? wkeys.wk_ring : wkeys.nwin;
+    w.lo = ring ? wkeys.lo_ring : 0;
+    w.nk = w.wk + w.j0 + w.nr;
+    w.ntiles = (w.nk + kWinKeys - 1) / kWinKeys;
+    return w;
+}
+
+// Window key `key` (< wk) of a unit holds a position inside the window.
+__device__ __forceinline__ bool win_valid(const WinUnit& w, const WinKeys& k, int R, int Wcap, int key) {
+    if (w.depth >= R) return true;
+    int d = w.lo + key - k.slot0;
+    if (d < 0) d += Wcap;
+    return d < k.nwin;
+}
+
+// One row's merge: deep splits 0..np-1 in order, then the window partial
+// (segment nsplit): M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L.  Eight
+// lanes per row (lane sl holds channels 4*sl + 32*c); every load is issued before
+// the arithmetic (one round trip).  NU >= np + 1 bounds the segments.
+template <int D, int NU>
+__device__ __forceinline__ void merge_row(const VerifyArgs& a, int64_t ro, int np, int sl) {
+    using sm100::ex2;
+    using sm100::pack_bf16;
+    constexpr int CH = D / 32;
+    const int64_t base = ro * a.nseg;
+    float2 ml[NU];
+    float4 x[NU][CH];
+#pragma unroll
+    for (int sg = 0; sg < NU; ++sg) {
+        if (sg <= np) {
+            const int64_t seg = base + (sg < np ? sg : a.nsplit);
+            ml[sg] = __ldcg(a.part_ml + seg);
+#pragma unroll
+            for (int c = 0; c < CH; ++c)
+                x[sg][c] = __ldcg(reinterpret_cast<const float4*>(a.part_o + seg * D + 4 * sl + 32 * c));
+        }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int sg = 0; sg < NU; ++sg)
+        if (sg <= np) M = fmaxf(M, ml[sg].x);
+    float f[NU], L = 0.f;
+#pragma unroll
+    for (int sg = 0; sg < NU; ++sg) {
+        if (sg <= np) {
+            f[sg] = ex2(ml[sg].x - M);
+            L = fmaf(ml[sg].y, f[sg], L);
+        }
+    }
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int sg = 0; sg < NU; ++sg) {
+            if (sg <= np) {
+                acc[0] = fmaf(x[sg][c].x, f[sg], acc[0]);
+                acc[1] = fmaf(x[sg][c].y, f[sg], acc[1]);
+                acc[2] = fmaf(x[sg][c].z, f[sg], acc[2]);
+                acc[3] = fmaf(x[sg][c].w, f[sg], acc[3]);
+            }
+        }
+        *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
+            make_uint2(pack_bf16(acc[0] / L, acc[1] / L), pack_bf16(acc[2] / L, acc[3] / L));
+    }
+    if (sl == 0 && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
+}
+
+// The same merge for any number of deep splits, one segment at a time (the same
+// operation order, so the same result).
+template <int D>
+__device__ __noinline__ void merge_row_any(const VerifyArgs& a, int64_t ro, int np, int sl) {
+    using sm100::ex2;
+    using sm100::pack_bf16;
+    constexpr int CH = D / 32;
+    const int64_t base = ro * a.nseg;
+    float M = -INFINITY;
+    for (int sg = 0; sg <= np; ++sg) M = fmaxf(M, __ldcg(a.part_ml + base + (sg < np ? sg : a.nsplit)).x);
+    float L = 0.f, acc[CH][4];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
+    for (int sg = 0; sg <= np; ++sg) {
+        const int64_t seg = base + (sg < np ? sg : a.nsplit);
+        const float2 ml = __ldcg(a.part_ml + seg);
+        const float f = ex2(ml.x - M);
+        L = fmaf(ml.y, f, L);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(a.part_o + seg * D + 4 * sl + 32 * c));
+            acc[c][0] = fmaf(x.x, f, acc[c][0]);
+            acc[c][1] = fmaf(x.y, f, acc[c][1]);
+            acc[c][2] = fmaf(x.z, f, acc[c][2]);
+            acc[c][3] = fmaf(x.w, f, acc[c][3]);
+        }
+    }
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D;
+#pragma unroll
+    for (int c = 0; c < CH; ++c)
+        *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
+            make_uint2(pack_bf16(acc[c][0] / L, acc[c][1] / L), pack_bf16(acc[c][2] / L, acc[c][3] / L));
+    if (sl == 0 && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
+}
+
+template <int D, int MT, int ST, int NW, int NS>
+__global__ void __launch_bounds__(FusedLayout<D, MT, ST, NW, NS>::THREADS, 1)
+verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, VerifyArgs a) {
+    using Lay = FusedLayout<D, MT, ST, NW, NS>;
+    using namespace sm100;
+    constexpr int NCH = Lay::NCH;
+    constexpr int RT = 128 * MT;
+    constexpr uint32_t IDESC_QK = idesc_bf16(128, kN, 0);
+    constexpr uint32_t IDESC_PV = idesc_bf16(128, D, 1);
+    constexpr int NWARPS = Lay::THREADS / 32;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = sm + Lay::OFF_Q;
+    uint8_t* sK = sm + Lay::OFF_K;
+    uint8_t* sV = sm + Lay::OFF_V;
+    uint8_t* sP = sm + Lay::OFF_P;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* v_full = bars + 1 + ST;
+    uint64_t* kv_empty = bars + 1 + 2 * ST;
+    uint64_t* s_full = bars + 1 + 3 * ST;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* pv_done = s_full + 4;
+    uint64_t* drain = s_full + 6;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 4);
+    GroupInfo* gi = reinterpret_cast<GroupInfo*>(sm + Lay::OFF_MISC + 16);
+    BranchEnt* bt = reinterpret_cast<BranchEnt*>(sm + Lay::OFF_BT);
+
+    const StoreView& s = a.s;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int g = blockIdx.x, h = blockIdx.y, split = blockIdx.z;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 128);
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(k_full + i, 1);
+            mbar_init(v_full + i, 1);
+            mbar_init(kv_empty + i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s_full + i, 1);
+            mbar_init(p_full + i, 128);
+            mbar_init(pv_done + i, 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, Lay::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // Inputs and scratch may belong to the previous kernel in the stream.
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    // ---- the group of branches this CTA serves (one sequence), its key range and units
+    if (warp == 0) {
+        int first, end;
+        if (a.ba.table) {
+            first = group_start(a.ba.table, a.ba.nbranch, g, lane);
+            end = first < a.ba.nbranch ? group_start(a.ba.table, a.ba.nbranch, g + 1, lane) : first;
+        } else {
+            first = min(g * s.R, a.ba.nbranch);
+            end = min(first + s.R, a.ba.nbranch);
+        }
+        int nb = end - first;
+        if (nb > kMaxGroupBranches) {
+            if (lane == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
+            nb = 0;
+        }
+        // Branch entries loaded in parallel; row and unit offsets by warp prefix sums.
+        int seq = -1, base = 0, ubase = 0;
+        for (int c0 = 0; c0 < nb; c0 += 32) {
+            const int i = c0 + lane;
+            Branch br;
+            br.ok = false;
+            if (i < nb) br = load_branch(a.ba, s.R, s.Bmax, first + i);
+            if (i < nb && !br.ok && split == 0 && h == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
+            const int n = (i < nb && br.ok) ? br.ntok : 0;
+            const int nu = (n + kWinRows - 1) / kWinRows;
+            int incl = n, uincl = nu;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                const int uy = __shfl_up_sync(0xffffffffu, uincl, o);
+                if (lane >= o) {
+                    incl += y;
+                    uincl += uy;
+                }
+            }
+            if (i < nb) bt[i] = BranchEnt{br.row0, br.stride, n, base + incl - n, br.depth, ubase + uincl - nu};
+            const unsigned okm = __ballot_sync(0xffffffffu, i < nb && br.ok);
+            if (seq < 0 && okm) seq = __shfl_sync(0xffffffffu, br.seq, __ffs(okm) - 1);
+            base += __shfl_sync(0xffffffffu, incl, 31);
+            ubase += __shfl_sync(0xffffffffu, uincl, 31);
+        }
+        if (lane == 0) {
+            GroupInfo info{first, nb, seq, base, 0, 0, 0, 0, ubase};
+            if (seq >= 0 && base > 0) {
+                info.T = context_length(s.len, a.ctx, s.err, seq, split == 0 && h == 0);
+                info.A = min(s.ws[seq], info.T);
+                info.key_begin = split * a.chunk;
+                info.key_end = min(info.A, info.key_begin + a.chunk);
+            } else {
+                info.nrows = 0;
+                info.units = 0;
+            }
+            if (g == gridDim.x - 1 && a.ba.table && end < a.ba.nbranch)
+                set_device_error(s.err, RIPE_DEVERR_BRANCH);  // more runs of sequences than CTAs
+            *gi = info;
+        }
+    }
+    __syncthreads();
+    const GroupInfo G = *gi;
+    const int ntiles = G.key_end > G.key_begin ? (G.key_end - G.key_begin + kN - 1) / kN : 0;
+    const int nrt = (G.nrows + RT - 1) / RT;
+    const int total_it = ntiles * nrt;
+
+    if (warp < 6) {
+        if (total_it > 0) {
+            if (warp == 4) {
+                // ------------------------------------------------ TMA producer
+                if (lane == 0) {
+                    const int row_base = ((a.layer * s.Bmax + G.seq) * s.H + h) * s.Tmax + G.key_begin;
+                    int issued = 0;
+                    for (int it = 0; it < total_it; ++it) {
+                        const int i = it % ntiles, st = it % ST;
+                        if (it >= ST && !mbar_wait(kv_empty + st, ((it / ST) - 1) & 1, abort_flag, s.err)) break;
+                        issued = it + 1;
+                        const int y = row_base + i * kN;
+                        mbar_expect_tx(k_full + st, Lay::KV_STAGE);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c)
+                            tma_load_2d(sK + st * Lay::KV_STAGE + c * 4096, &tmK, 32 * c, y, k_full + st);
+                        mbar_expect_tx(v_full + st, Lay::KV_STAGE);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c)
+                            tma_load_2d(sV + st * Lay::KV_STAGE + c * 4096, &tmV, 32 * c, y, v_full + st);
+                    }
+                    if (*abort_flag) {
+                        // Let the copies already issued land before the CTA's shared memory goes away.
+                        volatile int no_abort = 0;
+                        for (int it = issued > ST ? issued - ST : 0; it < issued; ++it) {
+                            mbar_wait(k_full + it % ST, (it / ST) & 1, &no_abort, s.err);
+                            mbar_wait(v_full + it % ST, (it / ST) & 1, &no_abort, s.err);
+                        }
+                    }
+                }
+            } else if (warp == 5) {
+                // ------------------------------------------------ MMA issuer
+                if (lane == 0) {
+                    const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV), p0 = smem_u32(sP);
+                    auto issue_pv = [&](int t) -> bool {
+                        const int st = t % ST, pb = t & 1, it_in_rt = t % ntiles;
+                        if (!mbar_wait(p_full + pb, (t >> 1) & 1, abort_flag, s.err)) return false;
+                        if (!mbar_wait(v_full + st, (t / ST) & 1, abort_flag, s.err)) return false;
+                        tc_fence_after();
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                            for (int ks = 0; ks < kN / 16; ++ks) {
+                                const uint64_t ad = smem_desc(p0 + (pb * MT + mt) * Lay::P_BUF + (ks >> 1) * 8192 +
+                                                                  (ks & 1) * 32, 16, 512, kLayoutSwizzle64B);
+                                const uint64_t bd = smem_desc(v0 + st * Lay::KV_STAGE + ks * 1024, kN * 64, 512,
+                                                              kLayoutSwizzle64B);
+                                mma_bf16(tmem + Lay::O_COL(mt), ad, bd, IDESC_PV,
+                                         (it_in_rt > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(kv_empty + st);
+                        mma_commit(pv_done + pb);
+                        return true;
+                    };
+                    bool ok = true;
+                    for (int it = 0; it < total_it && ok; ++it) {
+                        const int i = it % ntiles, st = it % ST, sb = it & 1;
+                        if (i == 0) {
+                            // A new row tile: finish the previous one before waiting for its Q.
+                            if (it > 0 && !(ok = issue_pv(it - 1))) break;
+                            if (!mbar_wait(q_full, (it / ntiles) & 1, abort_flag, s.err)) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!mbar_wait(k_full + st, (it / ST) & 1, abort_flag, s.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks & 1) * 32;
+                                const uint64_t ad = smem_desc(q0 + mt * NCH * 8192 + (ks >> 1) * 8192 + off, 16,
+                                                              512, kLayoutSwizzle64B);
+                                const uint64_t bd = smem_desc(k0 + st * Lay::KV_STAGE + (ks >> 1) * 4096 + off, 16,
+                                                              512, kLayoutSwizzle64B);
+                                mma_bf16(tmem + Lay::S_COL(mt, sb), ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(s_full + sb);
+                        if (i > 0) ok = issue_pv(it - 1);
+                    }
+                    if (ok) issue_pv(total_it - 1);
+                    // Every MMA issued so far has completed before TMEM is released.
+                    volatile int no_abort = 0;
+                    mma_commit(drain);
+                    mbar_wait(drain, 0, &no_abort, s.err);
+                }
+            } else {
+                // ------------------------------------------------ softmax + epilogue (warps 0-3)
+                const int t = threadIdx.x;  // TMEM lane / row within an M tile
+                const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+                const float c2 = a.scale_log2;
+                float m[MT], l[MT];
+                int rows[MT];
+                bool ok = true;
+                for (int it = 0; it < total_it && ok; ++it) {
+                    const int i = it % ntiles, rt = it / ntiles, sb = it & 1;
+                    if (i == 0) {
+                        // Rows of this row tile (each thread finds its own); the warp copies
+                        // its 32 rows' Q, 16 bytes per lane in row order (coalesced), into
+                        // the swizzled K-major layout.
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const int row = group_row(bt, G.nb, rt * RT + mt * 128 + t);
+                            rows[mt] = row;
+                            constexpr int QV = 2 * D / 16;  // 16-byte vectors per row
+#pragma unroll
+                            for (int e0 = 0; e0 < 32 * QV; e0 += 32) {
+                                const int e = e0 + lane, r = e / QV, v = e - r * QV;
+                                const int rrow = __shfl_sync(0xffffffffu, row, r);
+                                const int tr = warp * 32 + r;  // TMEM lane / row within the M tile
+                                uint8_t* dst = sQ + mt * NCH * 8192 + (v >> 2) * 8192 + tr * 64 +
+                                               (((v & 3) ^ ((tr >> 1) & 3)) << 4);
+                                const char* src =
+                                    rrow >= 0 ? a.Q + ((int64_t)rrow * s.H + h) * D * 2 + v * 16 : a.Q;
+                                cp_async16_zfill(dst, src, rrow >= 0);
+                            }
+                            m[mt] = -INFINITY;
+                            l[mt] = 0.f;
+                        }
+                        cp_async_commit();
+                        cp_async_wait_all();
+                        fence_proxy_async_smem();
+                        mbar_arrive(q_full);
+                    }
+                    if (!warp_wait(s_full + sb, (it >> 1) & 1, abort_flag, s.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int key0 = G.key_begin + i * kN;
+                    const int nvalid = min(kN, G.key_end - key0);
+                    if (it >= 2 && !warp_wait(pv_done + sb, ((it - 2) >> 1) & 1, abort_flag, s.err)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        float sc[kN];
+                        tmem_ld32(lane_addr + Lay::S_COL(mt, sb), sc);
+                        tmem_ld32(lane_addr + Lay::S_COL(mt, sb) + 32, sc + 32);
+                        tmem_wait_ld();
+                        if (nvalid < kN) {
+#pragma unroll
+                            for (int c = 0; c < kN; ++c)
+                                if (c >= nvalid) sc[c] = -INFINITY;
+                        }
+                        // Row max of the raw scores (scale > 0 commutes with max), four chains.
+                        float m4[4] = {sc[0], sc[1], sc[2], sc[3]};
+#pragma unroll
+                        for (int c = 4; c < kN; c += 4) {
+                            m4[0] = fmaxf(m4[0], sc[c]);
+                            m4[1] = fmaxf(m4[1], sc[c + 1]);
+                            m4[2] = fmaxf(m4[2], sc[c + 2]);
+                            m4[3] = fmaxf(m4[3], sc[c + 3]);
+                        }
+                        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
+                        // The running max moves only when it grows by more than 2^8 (probabilities
+                        // then stay below 256); the O rescale is warp-collective.
+                        float alpha = 1.f;
+                        const bool grow = mx > m[mt] + 8.f;
+                        if (grow) {
+                            const float mn = fmaxf(mx, m[mt]);
+                            alpha = ex2(m[mt] - mn);
+                            m[mt] = mn;
+                        }
+                        if (i > 0 && __any_sync(0xffffffffu, grow)) {
+                            // O holds this row tile's earlier tiles: rescale it once PV(it-1) is done.
+                            if (!warp_wait(pv_done + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, s.err)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+#pragma unroll
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                float o[32];
+                                tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int c = 0; c < 32; ++c) o[c] *= alpha;
+                                tmem_st32(lane_addr + Lay::O_COL(mt) + c0, o);
+                            }
+                            tmem_wait_st();
+                        }
+                        // p = 2^(s*scale*log2e - m): one FMA and one ex2 per score.
+                        const float nm = -m[mt];
+                        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                        uint8_t* prow = sP + (sb * MT + mt) * Lay::P_BUF + t * 64;
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+                            for (int gq = 0; gq < 4; ++gq) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float x0 = ex2(fmaf(sc[c * 32 + gq * 8 + 2 * e], c2, nm));
+                                    const float x1 = ex2(fmaf(sc[c * 32 + gq * 8 + 2 * e + 1], c2, nm));
+                                    s4[e] += x0 + x1;
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                                    w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                                }
+                                *reinterpret_cast<uint4*>(prow + c * 8192 + ((gq ^ ((t >> 1) & 3)) << 4)) =
+                                    make_uint4(w[0], w[1], w[2], w[3]);
+                            }
+                        }
+                        l[mt] = l[mt] * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                    }
+                    if (!ok) break;
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(p_full + sb);
+                    if (i == ntiles - 1) {
+                        // Row-tile epilogue: the partial (m, l, o) of every real row.
+                        if (!warp_wait(pv_done + sb, (it >> 1) & 1, abort_flag, s.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // The P buffers are free here (every PV of the row tile is done):
+                        // each warp stages 8 rows at a time there and stores them coalesced.
+                        constexpr int OSTR = 4 * D + 16;
+                        uint8_t* ostage = sP + warp * 8 * OSTR;
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const int row = rows[mt];
+                            float o[D];
+#pragma unroll
+                            for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o + c0);
+                            tmem_wait_ld();
+                            const int64_t pi = row >= 0 ? ((int64_t)row * s.H + h) * a.nseg + split : -1;
+                            if (row >= 0) a.part_ml[pi] = make_float2(m[mt], l[mt]);
+#pragma unroll
+                            for (int rr = 0; rr < 4; ++rr) {
+                                if ((lane >> 3) == rr) {
+                                    float4* d4 = reinterpret_cast<float4*>(ostage + (lane & 7) * OSTR);
+#pragma unroll
+                                    for (int c = 0; c < D / 4; ++c)
+                                        d4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                                }
+                                __syncwarp();
+#pragma unroll
+                                for (int e0 = 0; e0 < 8 * (D / 4); e0 += 32) {
+                                    const int e = e0 + lane, kr = e / (D / 4), c4 = e - kr * (D / 4);
+                                    const int64_t pk = __shfl_sync(0xffffffffu, pi, rr * 8 + kr);
+                                    if (pk >= 0)
+                                        reinterpret_cast<float4*>(a.part_o + pk * D)[c4] =
+                                            *reinterpret_cast<const float4*>(ostage + kr * OSTR + c4 * 16);
+                                }
+                                __syncwarp();
+                            }
+                        }
+                        tc_fence_before();
+                    }
+                }
+            }
+        }
+    } else if (G.units > 0) {
+        // ------------------------------------------------ window warps
+        constexpr int WSTR = Lay::WSTR;
+        constexpr int NV = 2 * D / 16;  // 16-byte vectors per row
+        constexpr int NKS = D / 16;     // k-steps of S^T = K Q^T
+        constexpr int NMT = D / 16;     // 16-channel tiles of O^T
+        const int ww = warp - 6;
+        uint8_t* wbuf = sm + Lay::OFF_W + ww * NS * Lay::WSTAGE;
+        const uint32_t wbuf_a = smem_u32(wbuf);
+        const WinKeys wkeys = win_keys(G.A, G.T, s.Wcap);
+        const int ustep = a.nsplit * NW;
+        const int nunits = G.units;
+        const float c2 = a.scale_log2;
+        const int64_t ring0 = ring_row(s, a.layer, G.seq, h, 1, 0);  // plane 1, slot 0
+        const int64_t plane_bytes = (int64_t)s.Wcap * 2 * D;        // one ring plane
+        const int64_t deep0 = deep_row(s, a.layer, G.seq, h, G.A);  // first window row of plane R
+        int iu = split + a.nsplit * ww;  // this warp's units: iu, iu + ustep, ...
+        if (iu < nunits) {
+            // Copies of tile t of unit w into stage `stage`: 16-byte vectors in row
+            // order (a warp instruction covers 512 contiguous bytes of window rows);
+            // keys outside the window or past the unit's keys are zero-filled.
+            auto issue = [&](const WinUnit& w, int t, int stage) {
+                uint8_t* sb = wbuf + stage * Lay::WSTAGE;
+                const bool ring = w.depth < s.R;
+                const int64_t wbase =
+                    ring ? ring0 + (int64_t)(w.depth - 1) * plane_bytes + (int64_t)w.lo * 2 * D : deep0;
+                const char* kw = (ring ? s.kwin : s.kdeep) + wbase;
+                const char* vw = (ring ? s.vwin : s.vdeep) + wbase;
+#pragma unroll
+                for (int e0 = 0; e0 < kWinKeys * NV; e0 += 32) {
+                    const int e = e0 + lane, kr = e / NV, v = e - kr * NV;
+                    const int key = t * kWinKeys + kr;
+                    const char* kp = a.Q;
+                    const char* vp = a.Q;
+                    bool ok;
+                    if (key < w.wk) {
+                        ok = win_valid(w, wkeys, s.R, s.Wcap, key);
+                        if (ok) {
+                            kp = kw + (int64_t)key * 2 * D + v * 16;
+                            vp = vw + (int64_t)key * 2 * D + v * 16;
+                        }
+                    } else {
+                        ok = key < w.nk;
+                        if (ok) {
+                            const int64_t off =
+                                (((int64_t)w.row0 + (int64_t)(key - w.wk) * w.stride) * s.H + h) * 2 * D + v * 16;
+                            kp = a.Kb + off;
+                            vp = a.Vb + off;
+                        }
+                    }
+                    cp_async16_zfill(sb + kr * WSTR + v * 16, kp, ok);
+                    cp_async16_zfill(sb + (kWinKeys + kr) * WSTR + v * 16, vp, ok);
+                }
+                if (t == 0) {
+#pragma unroll
+                    for (int e0 = 0; e0 < kWinRows * NV; e0 += 32) {
+                        const int e = e0 + lane, r = e / NV, v = e - r * NV;
+                        const bool okq = r < w.nr;
+                        const char* qp = okq ? a.Q + (((int64_t)w.row0 + (int64_t)(w.j0 + r) * w.stride) * s.H + h) *
+                                                         (2 * D) + v * 16
+                                             : a.Q;
+                        cp_async16_zfill(sb + (2 * kWinKeys + r) * WSTR + v * 16, qp, okq);
+                    }
+                }
+                cp_async_commit();
+            };
+
+            WinUnit wi = win_unit(bt, G.nb, iu, wkeys, s.R, lane);
+            WinUnit wc = wi;
+            int cu = iu, it_ = 0, ct = 0;
+            bool ihas = true;
+            auto advance_issue = [&]() {
+                if (++it_ == wi.ntiles) {
+                    iu += ustep;
+                    it_ = 0;
+                    if (iu < nunits)
+                        wi = win_unit(bt, G.nb, iu, wkeys, s.R, lane);
+                    else
+                        ihas = false;
+                }
+            };
+#pragma unroll
+            for (int sidx = 0; sidx < NS - 1; ++sidx) {
+                if (ihas) {
+                    issue(wi, it_, sidx);
+                    advance_issue();
+                } else {
+                    cp_async_commit();
+                }
+            }
+
+            uint32_t bq[NKS][2];
+            float o[NMT][4];
+            float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+            const int ra = 2 * (lane & 3), rb = ra + 1;  // fragment columns (rows) of this lane
+            const uint32_t k_lane = ((lane & 7) + 8 * ((lane >> 3) & 1)) * WSTR + 16 * (lane >> 4);
+            const uint32_t v_lane = kWinKeys * WSTR + ((lane & 7) + 8 * (lane >> 4)) * WSTR + 16 * ((lane >> 3) & 1);
+            const uint32_t q_lane = 2 * kWinKeys * WSTR + (lane & 7) * WSTR + 16 * (lane >> 3);
+            for (int q = 0;; ++q) {
+                if (ihas) {
+                    issue(wi, it_, (q + NS - 1) % NS);
+                    advance_issue();
+                } else {
+                    cp_async_commit();
+                }
+                cp_async_wait_group<NS - 1>();
+                __syncwarp();
+                const uint32_t sb = wbuf_a + (q % NS) * Lay::WSTAGE;
+                if (ct == 0) {
+                    // Q^T fragments (B operand, k-steps in pairs) and a fresh accumulator.
+#pragma unroll
+                    for (int s2 = 0; s2 < NKS / 2; ++s2)
+                        ldsm_x4(sb + q_lane + 64 * s2, bq[2 * s2][0], bq[2 * s2][1], bq[2 * s2 + 1][0],
+                                bq[2 * s2 + 1][1]);
+#pragma unroll
+                    for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+                    m_a = m_b = -INFINITY;
+                    l_a = l_b = 0.f;
+                }
+                // ---- S^T = K Q^T for 16 keys x 8 rows
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(sb + k_lane + 32 * ks, a0, a1, a2, a3);
+                    mma_16816(c, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+                }
+                // ---- visibility: window keys for every row, block token j' for rows j >= j'
+                const int k0 = ct * kWinKeys + (lane >> 2), k1 = k0 + 8;
+                const bool w0 = k0 < wc.wk && win_valid(wc, wkeys, s.R, s.Wcap, k0);
+                const bool w1 = k1 < wc.wk && win_valid(wc, wkeys, s.R, s.Wcap, k1);
+                auto vis = [&](int key, bool win, int r) {
+                    return r < wc.nr && key < wc.nk && (key < wc.wk ? win : key - wc.wk <= wc.j0 + r);
+                };
+                const float s0 = vis(k0, w0, ra) ? c[0] * c2 : -INFINITY;
+                const float s1 = vis(k0, w0, rb) ? c[1] * c2 : -INFINITY;
+                const float s2 = vis(k1, w1, ra) ? c[2] * c2 : -INFINITY;
+                const float s3 = vis(k1, w1, rb) ? c[3] * c2 : -INFINITY;
+                float mx_a = fmaxf(s0, s2), mx_b = fmaxf(s1, s3);
+#pragma unroll
+                for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, o2));
+                    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, o2));
+                }
+                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+                const float al_a = mn_a == -INFINITY ? 1.f : ex2(m_a - mn_a);
+                const float al_b = mn_b == -INFINITY ? 1.f : ex2(m_b - mn_b);
+                const float p0 = mn_a == -INFINITY ? 0.f : ex2(s0 - mn_a);
+                const float p1 = mn_b == -INFINITY ? 0.f : ex2(s1 - mn_b);
+                const float p2 = mn_a == -INFINITY ? 0.f : ex2(s2 - mn_a);
+                const float p3 = mn_b == -INFINITY ? 0.f : ex2(s3 - mn_b);
+                l_a = l_a * al_a + (p0 + p2);
+                l_b = l_b * al_b + (p1 + p3);
+                m_a = mn_a;
+                m_b = mn_b;
+                // ---- O^T += V^T P^T: P^T by an 8x8 transpose of the S^T fragments
+                const uint32_t b0 = movmatrix_t(pack_bf16(p0, p1));
+                const uint32_t b1 = movmatrix_t(pack_bf16(p2, p3));
+#pragma unroll
+                for (int mt = 0; mt < NMT; ++mt) {
+                    o[mt][0] *= al_a;
+                    o[mt][1] *= al_b;
+                    o[mt][2] *= al_a;
+                    o[mt][3] *= al_b;
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(sb + v_lane + 32 * mt, a0, a1, a2, a3);
+                    mma_16816(o[mt], a0, a1, a2, a3, b0, b1);
+                }
+                if (ct == wc.ntiles - 1) {
+                    // ---- the unit's partial: rows ra and rb of this lane's columns
+#pragma unroll
+                    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                        l_a += __shfl_xor_sync(0xffffffffu, l_a, o2);
+                        l_b += __shfl_xor_sync(0xffffffffu, l_b, o2);
+                    }
+                    const bool va = ra < wc.nr, vb = rb < wc.nr;
+                    const int64_t pa =
+                        (((int64_t)wc.row0 + (int64_t)(wc.j0 + ra) * wc.stride) * s.H + h) * a.nseg + a.nsplit;
+                    const int64_t pb =
+                        (((int64_t)wc.row0 + (int64_t)(wc.j0 + rb) * wc.stride) * s.H + h) * a.nseg + a.nsplit;
+#pragma unroll
+                    for (int mt = 0; mt < NMT; ++mt) {
+                        const int ch = 16 * mt + (lane >> 2);
+                        if (va) {
+                            a.part_o[pa * D + ch] = o[mt][0];
+                            a.part_o[pa * D + ch + 8] = o[mt][2];
+                        }
+                        if (vb) {
+                            a.part_o[pb * D + ch] = o[mt][1];
+                            a.part_o[pb * D + ch + 8] = o[mt][3];
+                        }
+                    }
+                    if (lane < 4) {
+                        if (va) a.part_ml[pa] = make_float2(m_a, l_a);
+                        if (vb) a.part_ml[pb] = make_float2(m_b, l_b);
+                    }
+                }
+                __syncwarp();
+                if (++ct == wc.ntiles) {
+                    cu += ustep;
+                    if (cu >= nunits) break;
+                    wc = win_unit(bt, G.nb, cu, wkeys, s.R, lane);
+                    ct = 0;
+                }
+            }
+            cp_async_wait_all();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, Lay::TMEM_COLS);
+
+    // ---- merge: every partial of the cluster is written; this CTA merges rows
+    // split, split + nsplit, ... (8 lanes per row, four rows per warp at a time).
+    if (a.nsplit > 1) cluster_sync_all();
+    if (G.nrows > 0 && !*abort_flag) {
+        const int np = deep_splits_used(G.A, a.chunk, a.nsplit);
+        const int sub = lane >> 3, sl = lane & 7;
+        for (int k = warp * 4; split + a.nsplit * k < G.nrows; k += NWARPS * 4) {
+            const int rl = split + a.nsplit * (k + sub);
+            const int row = rl < G.nrows ? group_row(bt, G.nb, rl) : -1;
+            if (row < 0) continue;
+            const int64_t ro = (int64_t)row * s.H + h;
+            if (np < 4)
+                merge_row<D, 4>(a, ro, np, sl);
+            else
+                merge_row_any<D>(a, ro, np, sl);
+        }
+    }
+}
+
+template <int D, int MT, int ST, int NW, int NS>
+cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyArgs& a, int gslots, bool pdl,
+                     cudaStream_t st) {
+    using Lay = FusedLayout<D, MT, ST, NW, NS>;
+    static_assert(Lay::SMEM <= 232448, "shared memory budget");
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(verify_kernel<D, MT, ST, NW, NS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(verify_kernel<D, MT, ST, NW, NS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gslots, a.s.H, a.nsplit);
+    cfg.blockDim = dim3(Lay::THREADS);
+    cfg.dynamicSmemBytes = Lay::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (a.nsplit > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = 1;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = a.nsplit;
+        ++n;
+    }
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, verify_kernel<D, MT, ST, NW, NS>, tk, tv, a);
+    ripe_count_launch();
+    return e;
+}
+
+}  // namespace
+
+bool fused_supported(int dtype, int d) { return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128); }
+
+cudaError_t launch_fused(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt, bool pdl,
+                         cudaStream_t st) {
+    const CUtensorMap& tk = *reinterpret_cast<const CUtensorMap*>(tmK);
+    const CUtensorMap& tv = *reinterpret_cast<const CUtensorMap*>(tmV);
+    const int d = a.s.d;
+    // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
+    if (mt == 1) {
+        if (d == 64) return launch_t<64, 1, 4, 4, 3>(tk, tv, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 1, 2, 4, 3>(tk, tv, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 1, 2, 4, 2>(tk, tv, a, gslots, pdl, st);
+    } else {
+        if (d == 64) return launch_t<64, 2, 3, 4, 3>(tk, tv, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 2, 2, 3, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 2, 2, 1, 2>(tk, tv, a, gslots, pdl, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// Tensor maps of the deep planes: 2-D [rows = L*Bmax*H*Tmax][d] bf16, box 32 x 64
+// with the 64-byte swizzle the MMA descriptors above expect.
+int make_deep_tensor_maps(ripe_cache_s* c) {
+    typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return -1;
+        encode = reinterpret_cast<EncodeFn>(fn);
+    }
+    const cuuint64_t rows = (cuuint64_t)c->L * c->Bmax * c->H * c->Tmax;
+    if (rows >= (1ull << 31)) return -2;
+    const cuuint64_t dims[2] = {(cuuint64_t)c->d, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)c->d * 2};
+    const cuuint32_t box[2] = {32, (cuuint32_t)kN};
+    const cuuint32_t estr[2] = {1, 1};
+    CUtensorMap* maps[2] = {reinterpret_cast<CUtensorMap*>(c->tmap_k), reinterpret_cast<CUtensorMap*>(c->tmap_v)};
+    void* bases[2] = {c->kdeep, c->vdeep};
+    for (int i = 0; i < 2; ++i) {
+        CUresult r = encode(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, bases[i], dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return -3;
+    }
+    return 0;
+}

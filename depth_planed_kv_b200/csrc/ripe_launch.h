@@ -20,29 +20,22 @@ cudaError_t launch_synth_fill(const ripe_cache_s* c, int b, int T, uint64_t seed
 struct VerifyPlan {
     int nsplit;        // deep-region splits (partials 0..nsplit-1); the window+block partial is nsplit
     int chunk;         // keys per deep split
-    int rows_chunk;    // rows per CTA of the window kernel
-    int nrowchunks;    // row chunks per branch
+    int nrowchunks;    // row chunks per branch (CUDA-core kernel)
     int max_ntok;      // host bound on tokens per branch
-    bool tc_deep;      // deep region on the tcgen05 stacked-query kernel
-    int mt;            // M tiles (of 128 rows) per deep CTA
-    int gslots;        // deep CTAs along the sequence-group axis
+    bool fused;        // the whole call in the sm_100a fused kernel (tcgen05 deep region)
+    int mt;            // M tiles (of 128 rows) per fused CTA
+    int gslots;        // fused CTAs along the sequence-group axis
     size_t work_bytes; // scratch needed
-    int64_t counters;  // arrival counters the call uses (branches x row chunks x heads)
 };
 
-// Arrival counters available in a verify scratch.
-int64_t verify_max_counters();
-
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths);
+// Re-plan with `nsplit` deep splits (chunk and scratch size follow).
+void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit);
 
 struct VerifyArgs;
-bool deep_tc_supported(int dtype, int d);
-cudaError_t launch_deep_tc(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt, bool pdl,
-                           cudaStream_t st);
-bool window_supported(int dtype, int d);
-cudaError_t launch_window(const VerifyArgs& a, int nbranch, int keys_ub, bool pdl, cudaStream_t st);
-// Zero the arrival counters of a verify scratch (after a device error left them set).
-cudaError_t reset_verify_counters(void* work, cudaStream_t st);
+bool fused_supported(int dtype, int d);
+cudaError_t launch_fused(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt, bool pdl,
+                         cudaStream_t st);
 int make_deep_tensor_maps(ripe_cache_s* c);
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
@@ -51,7 +44,3 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
 
 // Record a one-line message for ripe_last_error() and return `status`.
 int ripe_fail(int status, const char* fmt, ...);
-
-// Zero the arrival counters of the allocation-free entry point's fixed scratch
-// (no-op if it was never used on the current device).
-cudaError_t reset_noalloc_counters(cudaStream_t st);

@@ -51,18 +51,6 @@ cudaError_t static_scratch_address(void** out) {
 
 }  // namespace
 
-cudaError_t reset_noalloc_counters(cudaStream_t st) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return e;
-    void* p = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        p = g_scratch_addr[dev];
-    }
-    return reset_verify_counters(p, st);
-}
-
 extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_branch_t* branches, int nbranch,
                                         int nrows, const void* Q, const void* Kb, const void* Vb,
                                         const int32_t* ctx, float scale, void* O, float* lse,
@@ -85,18 +73,8 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
     ba.nrows = nrows;
     ba.max_ntok = c->kmax;
     VerifyPlan plan = plan_verify(c, nbranch, nrows, c->kmax, false);
-    if (plan.counters > verify_max_counters())
-        return ripe_fail(RIPE_ERR_CAPACITY, "%lld (branch, row chunk, head) units in one call; at most %lld",
-                         (long long)plan.counters, (long long)verify_max_counters());
     // Fewer, longer deep splits until the partial results fit the fixed array.
-    while (plan.work_bytes > kStaticScratchBytes && plan.nsplit > 1) {
-        plan.nsplit = plan.nsplit / 2;
-        const int A_ub = c->len_ub < c->Tmax ? c->len_ub : c->Tmax;
-        int chunk = (A_ub + plan.nsplit - 1) / plan.nsplit;
-        chunk = (chunk + 31) / 32 * 32;
-        plan.chunk = chunk < 32 ? 32 : chunk;
-        plan.work_bytes = verify_work_bytes(nrows, c->H, c->d, plan.nsplit + 1);
-    }
+    while (plan.work_bytes > kStaticScratchBytes && plan.nsplit > 1) plan_set_splits(plan, c, nrows, plan.nsplit / 2);
     if (scratch_needed) *scratch_needed = plan.work_bytes;
     if (plan.work_bytes > kStaticScratchBytes)
         return ripe_fail(RIPE_ERR_CAPACITY, "this call needs %zu bytes of scratch; the static scratch holds %zu",

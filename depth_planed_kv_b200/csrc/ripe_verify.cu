@@ -395,27 +395,20 @@ cudaError_t launch_seg(const VerifyArgs& a, int seg_first, int seg_count, int nb
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths) {
     VerifyPlan p{};
     p.max_ntok = max_ntok;
-    p.rows_chunk = kRowsPerCta;
     p.nrowchunks = (max_ntok + kRowsPerCta - 1) / kRowsPerCta;
     if (p.nrowchunks < 1) p.nrowchunks = 1;
     const int A_ub = c->len_ub < c->Tmax ? c->len_ub : c->Tmax;
-    p.tc_deep = c->tc_ready && deep_tc_supported(c->dtype, c->d);
+    p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
     int64_t ns;
-    if (p.tc_deep) {
-        // One deep CTA per (sequence group, head, split); splits only until the
-        // CTAs cover the 148 SMs once (each CTA holds one SM's tensor memory).
+    if (p.fused) {
+        // One CTA per (sequence group, head, split); splits (a cluster, at most 8)
+        // only until the CTAs cover the 148 SMs once: each CTA holds one SM.
         p.gslots = all_depths ? nbranch / c->R : (nbranch < c->Bmax ? nbranch : c->Bmax);
         p.mt = (all_depths && max_ntok * c->R > 128) ? 2 : 1;
         const int64_t units = (int64_t)p.gslots * c->H;
         ns = units > 0 ? 148 / units : 1;
-        int64_t max_ns = (A_ub + 255) / 256;
-        if (max_ns > 8) max_ns = 8;  // the deep-side merge combines at most 8 deep partials
-        if (ns > max_ns) ns = max_ns;
+        if (ns > 8) ns = 8;
         if (ns < 1) ns = 1;
-        p.nsplit = (int)ns;
-        int chunk = (int)((A_ub + ns - 1) / ns);
-        chunk = (chunk + 63) / 64 * 64;
-        p.chunk = chunk < 64 ? 64 : chunk;
     } else {
         const int64_t items = (int64_t)nbranch * p.nrowchunks * c->H;
         const int64_t target = 148 * 8;
@@ -423,22 +416,21 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
         const int64_t max_ns = (A_ub + 63) / 64;
         if (ns > max_ns) ns = max_ns;
         if (ns < 1) ns = 1;
-        p.nsplit = (int)ns;
-        int chunk = (int)((A_ub + ns - 1) / ns);
-        chunk = (chunk + 31) / 32 * 32;
-        p.chunk = chunk < 32 ? 32 : chunk;
         p.mt = 0;
         p.gslots = 0;
     }
-    p.work_bytes = verify_work_bytes(nrows, c->H, c->d, p.nsplit + 1);
-    p.counters = (int64_t)nbranch * p.nrowchunks * c->H;
+    plan_set_splits(p, c, nrows, (int)ns);
     return p;
 }
 
-int64_t verify_max_counters() { return kMaxCounters; }
-
-cudaError_t reset_verify_counters(void* work, cudaStream_t st) {
-    return work ? cudaMemsetAsync(work, 0, kCounterBytes, st) : cudaSuccess;
+void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit) {
+    const int A_ub = c->len_ub < c->Tmax ? c->len_ub : c->Tmax;
+    const int align = p.fused ? 64 : 32;  // deep tile of the fused kernel / key tile of the CUDA-core kernel
+    p.nsplit = nsplit;
+    int chunk = (A_ub + nsplit - 1) / nsplit;
+    chunk = (chunk + align - 1) / align * align;
+    p.chunk = chunk < align ? align : chunk;
+    p.work_bytes = verify_work_bytes(nrows, c->H, c->d, nsplit + 1);
 }
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
@@ -454,18 +446,14 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     a.nsplit = plan.nsplit; a.chunk = plan.chunk; a.nseg = plan.nsplit + 1;
     a.nrowchunks = plan.nrowchunks;
     char* wb = reinterpret_cast<char*>(work);
-    a.cnt = reinterpret_cast<int*>(wb);
-    a.done = reinterpret_cast<int*>(wb + kCounterBytes - 256);
-    a.part_ml = reinterpret_cast<float2*>(wb + kCounterBytes);
-    a.part_o = reinterpret_cast<float*>(wb + kCounterBytes + verify_ml_bytes(ba.nrows, c->H, a.nseg));
+    a.part_ml = reinterpret_cast<float2*>(wb);
+    a.part_o = reinterpret_cast<float*>(wb + verify_ml_bytes(ba.nrows, c->H, a.nseg));
     cudaError_t e;
     const int win_ub = (c->len_ub < c->Wcap ? c->len_ub : c->Wcap) + plan.max_ntok;
-    if (plan.tc_deep) {
-        // Deep region on the tensor cores and, beside it (programmatic dependent
-        // launch), the window/block kernel; the last contributor of a row merges.
-        e = launch_deep_tc(c->tmap_k, c->tmap_v, a, plan.gslots, plan.mt, true, st);
-        if (e != cudaSuccess) return e;
-        e = launch_window(a, ba.nbranch, win_ub, true, st);
+    if (plan.fused) {
+        // The whole call in one kernel; programmatic dependent launch lets its
+        // prologue overlap the tail of the previous kernel in the stream.
+        e = launch_fused(c->tmap_k, c->tmap_v, a, plan.gslots, plan.mt, true, st);
         if (e != cudaSuccess) return e;
     } else {
         const int keys_ub = plan.chunk > win_ub ? plan.chunk : win_ub;

@@ -16,8 +16,6 @@ struct VerifyArgs {
     int nrowchunks;           // row chunks per branch in the CUDA-core kernel
     float2* part_ml;          // [nrows][H][nseg] (m in log2 units, l)
     float* part_o;            // [nrows][H][nseg][d]
-    int* cnt;                 // [nbranch][H] arrivals of partials per (branch, head); self-resetting
-    int* done;                // CTAs of the window kernel that finished; self-resetting
 };
 
 // Deep splits that hold keys for a sequence whose deep region has A keys.
@@ -26,14 +24,10 @@ __host__ __device__ inline int deep_splits_used(int A, int chunk, int nsplit) {
     return n < nsplit ? n : nsplit;
 }
 
-// Scratch layout: a fixed region of arrival counters (they reset themselves and
-// must start at zero, so they never move), then the (m, l) pairs, padded to 256
-// bytes, then the o vectors.
-constexpr size_t kCounterBytes = size_t(1) << 20;
-constexpr int64_t kMaxCounters = (int64_t)(kCounterBytes - 256) / 4;  // the done counter sits at the end
+// Scratch layout: the (m, l) pairs, padded to 256 bytes, then the o vectors.
 inline size_t verify_ml_bytes(int nrows, int H, int nseg) {
     return ((size_t)nrows * H * nseg * sizeof(float2) + 255) / 256 * 256;
 }
 inline size_t verify_work_bytes(int nrows, int H, int d, int nseg) {
-    return kCounterBytes + verify_ml_bytes(nrows, H, nseg) + (size_t)nrows * H * nseg * d * sizeof(float);
+    return verify_ml_bytes(nrows, H, nseg) + (size_t)nrows * H * nseg * d * sizeof(float);
 }
