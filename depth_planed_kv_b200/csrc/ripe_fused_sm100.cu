@@ -48,6 +48,7 @@ constexpr int kDeepThreads = 192;  // warps 0-3 softmax, 4 TMA, 5 MMA
 constexpr int kMaxGroupBranches = 64;
 constexpr int kWinRows = 8;   // rows per window unit (the N of an m16n8k16 tile)
 constexpr int kWinKeys = 16;  // keys per window tile (the M of an m16n8k16 tile)
+constexpr int kRowTable = 512;  // group rows whose Q/O row index is tabulated in shared memory
 
 // One branch of the group: its rows, its offset among the group's rows, its
 // depth and the index of its first window unit.
@@ -77,7 +78,8 @@ struct FusedLayout {
     static constexpr int NBAR = 1 + 3 * ST + 7;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_BT = OFF_MISC + 64;
-    static constexpr int BYTES = OFF_BT + kMaxGroupBranches * (int)sizeof(BranchEnt);
+    static constexpr int OFF_RT = OFF_BT + kMaxGroupBranches * (int)sizeof(BranchEnt);
+    static constexpr int BYTES = OFF_RT + kRowTable * 4;
     static constexpr int SMEM = BYTES + 1024;  // alignment slack
     static constexpr int THREADS = kDeepThreads + 32 * NW;
     static constexpr uint32_t TMEM_COLS = MT == 1 ? 256 : 512;
@@ -93,10 +95,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Row (of Q/O) of the group's rl-th query, branches in table order; -1 past the end.
-__device__ int group_row(const BranchEnt* bt, int nb, int rl) {
+__device__ int group_row_scan(const BranchEnt* bt, int nb, int rl) {
     for (int i = 0; i < nb; ++i)
         if (rl < bt[i].off + bt[i].ntok) return bt[i].row0 + (rl - bt[i].off) * bt[i].stride;
     return -1;
+}
+// The same from the shared-memory row table for the first kRowTable rows.
+__device__ __forceinline__ int group_row(const int* rowtab, const BranchEnt* bt, int nb, int nrows, int rl) {
+    if (rl >= nrows) return -1;
+    return rl < kRowTable ? rowtab[rl] : group_row_scan(bt, nb, rl);
 }
 
 // Start of the g-th run of equal sequence ids in the branch table (warp-wide).
@@ -179,94 +186,104 @@ __device__ __forceinline__ bool win_valid(const WinUnit& w, const WinKeys& k, in
     return d < k.nwin;
 }
 
-// One row's merge: deep splits 0..np-1 in order, then the window partial
-// (segment nsplit): M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L.  Eight
-// lanes per row (lane sl holds channels 4*sl + 32*c); every load is issued before
-// the arithmetic (one round trip).  NU >= np + 1 bounds the segments.
-template <int D, int NU>
-__device__ __forceinline__ void merge_row(const VerifyArgs& a, int64_t ro, int np, int sl) {
+// The merge of NR rows (ro: row * H + head; ok: row exists): deep splits 0..np-1
+// in order, then the window partial (segment nsplit): M = max m,
+// L = sum l 2^(m-M), O = sum o 2^(m-M) / L.  Eight lanes per row (lane sl holds
+// channels 4*sl + 32*c); every load of the NR rows is issued before the
+// arithmetic (one round trip).  NU >= np + 1 bounds the segments.
+template <int D, int NU, int NR>
+__device__ __forceinline__ void merge_rows(const VerifyArgs& a, const int64_t* ro, const bool* ok, int np, int sl) {
     using sm100::ex2;
     using sm100::pack_bf16;
     constexpr int CH = D / 32;
-    const int64_t base = ro * a.nseg;
-    float2 ml[NU];
-    float4 x[NU][CH];
+    float2 ml[NR][NU];
+    float4 x[NR][NU][CH];
 #pragma unroll
-    for (int sg = 0; sg < NU; ++sg) {
-        if (sg <= np) {
-            const int64_t seg = base + (sg < np ? sg : a.nsplit);
-            ml[sg] = __ldcg(a.part_ml + seg);
+    for (int r = 0; r < NR; ++r) {
 #pragma unroll
-            for (int c = 0; c < CH; ++c)
-                x[sg][c] = __ldcg(reinterpret_cast<const float4*>(a.part_o + seg * D + 4 * sl + 32 * c));
+        for (int sg = 0; sg < NU; ++sg) {
+            if (ok[r] && sg <= np) {
+                const int64_t seg = ro[r] * a.nseg + (sg < np ? sg : a.nsplit);
+                ml[r][sg] = __ldcg(a.part_ml + seg);
+#pragma unroll
+                for (int c = 0; c < CH; ++c)
+                    x[r][sg][c] = __ldcg(reinterpret_cast<const float4*>(a.part_o + seg * D + 4 * sl + 32 * c));
+            }
         }
     }
-    float M = -INFINITY;
 #pragma unroll
-    for (int sg = 0; sg < NU; ++sg)
-        if (sg <= np) M = fmaxf(M, ml[sg].x);
-    float f[NU], L = 0.f;
+    for (int r = 0; r < NR; ++r) {
+        if (!ok[r]) continue;
+        float M = -INFINITY;
 #pragma unroll
-    for (int sg = 0; sg < NU; ++sg) {
-        if (sg <= np) {
-            f[sg] = ex2(ml[sg].x - M);
-            L = fmaf(ml[sg].y, f[sg], L);
-        }
-    }
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D;
-#pragma unroll
-    for (int c = 0; c < CH; ++c) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int sg = 0; sg < NU; ++sg)
+            if (sg <= np) M = fmaxf(M, ml[r][sg].x);
+        float f[NU], L = 0.f;
 #pragma unroll
         for (int sg = 0; sg < NU; ++sg) {
             if (sg <= np) {
-                acc[0] = fmaf(x[sg][c].x, f[sg], acc[0]);
-                acc[1] = fmaf(x[sg][c].y, f[sg], acc[1]);
-                acc[2] = fmaf(x[sg][c].z, f[sg], acc[2]);
-                acc[3] = fmaf(x[sg][c].w, f[sg], acc[3]);
+                f[sg] = ex2(ml[r][sg].x - M);
+                L = fmaf(ml[r][sg].y, f[sg], L);
             }
         }
-        *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
-            make_uint2(pack_bf16(acc[0] / L, acc[1] / L), pack_bf16(acc[2] / L, acc[3] / L));
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro[r] * D;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int sg = 0; sg < NU; ++sg) {
+                if (sg <= np) {
+                    acc[0] = fmaf(x[r][sg][c].x, f[sg], acc[0]);
+                    acc[1] = fmaf(x[r][sg][c].y, f[sg], acc[1]);
+                    acc[2] = fmaf(x[r][sg][c].z, f[sg], acc[2]);
+                    acc[3] = fmaf(x[r][sg][c].w, f[sg], acc[3]);
+                }
+            }
+            *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
+                make_uint2(pack_bf16(acc[0] / L, acc[1] / L), pack_bf16(acc[2] / L, acc[3] / L));
+        }
+        if (sl == 0 && a.lse) a.lse[ro[r]] = (M + log2f(L)) * 0.69314718055994531f;
     }
-    if (sl == 0 && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
 }
 
 // The same merge for any number of deep splits, one segment at a time (the same
 // operation order, so the same result).
 template <int D>
-__device__ __noinline__ void merge_row_any(const VerifyArgs& a, int64_t ro, int np, int sl) {
+__device__ __noinline__ void merge_row_any(const float2* part_ml, const float* part_o, char* O_, float* lse,
+                                           int nseg, int nsplit, int64_t ro, int np, int sl) {
     using sm100::ex2;
     using sm100::pack_bf16;
     constexpr int CH = D / 32;
-    const int64_t base = ro * a.nseg;
+    const int64_t base = ro * nseg;
     float M = -INFINITY;
-    for (int sg = 0; sg <= np; ++sg) M = fmaxf(M, __ldcg(a.part_ml + base + (sg < np ? sg : a.nsplit)).x);
+    for (int sg = 0; sg <= np; ++sg) M = fmaxf(M, __ldcg(part_ml + base + (sg < np ? sg : nsplit)).x);
     float L = 0.f, acc[CH][4];
 #pragma unroll
     for (int c = 0; c < CH; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
     for (int sg = 0; sg <= np; ++sg) {
-        const int64_t seg = base + (sg < np ? sg : a.nsplit);
-        const float2 ml = __ldcg(a.part_ml + seg);
+        const int64_t seg = base + (sg < np ? sg : nsplit);
+        const float2 ml = __ldcg(part_ml + seg);
         const float f = ex2(ml.x - M);
         L = fmaf(ml.y, f, L);
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-            const float4 x = __ldcg(reinterpret_cast<const float4*>(a.part_o + seg * D + 4 * sl + 32 * c));
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(part_o + seg * D + 4 * sl + 32 * c));
             acc[c][0] = fmaf(x.x, f, acc[c][0]);
             acc[c][1] = fmaf(x.y, f, acc[c][1]);
             acc[c][2] = fmaf(x.z, f, acc[c][2]);
             acc[c][3] = fmaf(x.w, f, acc[c][3]);
         }
     }
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(O_) + ro * D;
 #pragma unroll
     for (int c = 0; c < CH; ++c)
         *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
             make_uint2(pack_bf16(acc[c][0] / L, acc[c][1] / L), pack_bf16(acc[c][2] / L, acc[c][3] / L));
-    if (sl == 0 && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
+    if (sl == 0 && lse) lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
 }
 
+// One CTA per SM.  Registers come from the four SM sub-partitions (16384 each),
+// which hold ceil(warps / 4) warps apiece: 168 per thread for 9-12 warps.
 template <int D, int MT, int ST, int NW, int NS>
 __global__ void __launch_bounds__(FusedLayout<D, MT, ST, NW, NS>::THREADS, 1)
 verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, VerifyArgs a) {
@@ -297,6 +314,7 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 4);
     GroupInfo* gi = reinterpret_cast<GroupInfo*>(sm + Lay::OFF_MISC + 16);
     BranchEnt* bt = reinterpret_cast<BranchEnt*>(sm + Lay::OFF_BT);
+    int* rowtab = reinterpret_cast<int*>(sm + Lay::OFF_RT);
 
     const StoreView& s = a.s;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -370,7 +388,11 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     uincl += uy;
                 }
             }
-            if (i < nb) bt[i] = BranchEnt{br.row0, br.stride, n, base + incl - n, br.depth, ubase + uincl - nu};
+            if (i < nb) {
+                bt[i] = BranchEnt{br.row0, br.stride, n, base + incl - n, br.depth, ubase + uincl - nu};
+                for (int j = 0, rl = base + incl - n; j < n && rl < kRowTable; ++j, ++rl)
+                    rowtab[rl] = br.row0 + j * br.stride;
+            }
             const unsigned okm = __ballot_sync(0xffffffffu, i < nb && br.ok);
             if (seq < 0 && okm) seq = __shfl_sync(0xffffffffu, br.seq, __ffs(okm) - 1);
             base += __shfl_sync(0xffffffffu, incl, 31);
@@ -506,7 +528,7 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         // the swizzled K-major layout.
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
-                            const int row = group_row(bt, G.nb, rt * RT + mt * 128 + t);
+                            const int row = group_row(rowtab, bt, G.nb, G.nrows, rt * RT + mt * 128 + t);
                             rows[mt] = row;
                             constexpr int QV = 2 * D / 16;  // 16-byte vectors per row
 #pragma unroll
@@ -569,24 +591,6 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                             alpha = ex2(m[mt] - mn);
                             m[mt] = mn;
                         }
-                        if (i > 0 && __any_sync(0xffffffffu, grow)) {
-                            // O holds this row tile's earlier tiles: rescale it once PV(it-1) is done.
-                            if (!warp_wait(pv_done + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, s.err)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-#pragma unroll
-                            for (int c0 = 0; c0 < D; c0 += 32) {
-                                float o[32];
-                                tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int c = 0; c < 32; ++c) o[c] *= alpha;
-                                tmem_st32(lane_addr + Lay::O_COL(mt) + c0, o);
-                            }
-                            tmem_wait_st();
-                        }
                         // p = 2^(s*scale*log2e - m): one FMA and one ex2 per score.
                         const float nm = -m[mt];
                         float s4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -609,6 +613,25 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                             }
                         }
                         l[mt] = l[mt] * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                        if (i > 0 && __any_sync(0xffffffffu, grow)) {
+                            // O holds this row tile's earlier tiles: rescale it once PV(it-1) is done
+                            // (after P, so the scores no longer occupy registers).
+                            if (!warp_wait(pv_done + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, s.err)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+#pragma unroll
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                float o[32];
+                                tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int c = 0; c < 32; ++c) o[c] *= alpha;
+                                tmem_st32(lane_addr + Lay::O_COL(mt) + c0, o);
+                            }
+                            tmem_wait_st();
+                        }
                     }
                     if (!ok) break;
                     fence_proxy_async_smem();
@@ -622,33 +645,31 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         }
                         tc_fence_after();
                         // The P buffers are free here (every PV of the row tile is done):
-                        // each warp stages 8 rows at a time there and stores them coalesced.
-                        constexpr int OSTR = 4 * D + 16;
-                        uint8_t* ostage = sP + warp * 8 * OSTR;
+                        // each warp passes its 32 rows through them 32 columns at a time
+                        // and stores 128-byte row pieces (coalesced).
+                        constexpr int OSTR = 32 * 4 + 16;
+                        uint8_t* ostage = sP + warp * 32 * OSTR;
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             const int row = rows[mt];
-                            float o[D];
-#pragma unroll
-                            for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o + c0);
-                            tmem_wait_ld();
                             const int64_t pi = row >= 0 ? ((int64_t)row * s.H + h) * a.nseg + split : -1;
                             if (row >= 0) a.part_ml[pi] = make_float2(m[mt], l[mt]);
+#pragma unroll 1
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                float o[32];
+                                tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
+                                tmem_wait_ld();
+                                float4* d4 = reinterpret_cast<float4*>(ostage + lane * OSTR);
 #pragma unroll
-                            for (int rr = 0; rr < 4; ++rr) {
-                                if ((lane >> 3) == rr) {
-                                    float4* d4 = reinterpret_cast<float4*>(ostage + (lane & 7) * OSTR);
-#pragma unroll
-                                    for (int c = 0; c < D / 4; ++c)
-                                        d4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-                                }
+                                for (int c = 0; c < 8; ++c)
+                                    d4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
                                 __syncwarp();
 #pragma unroll
-                                for (int e0 = 0; e0 < 8 * (D / 4); e0 += 32) {
-                                    const int e = e0 + lane, kr = e / (D / 4), c4 = e - kr * (D / 4);
-                                    const int64_t pk = __shfl_sync(0xffffffffu, pi, rr * 8 + kr);
+                                for (int e0 = 0; e0 < 32 * 8; e0 += 32) {
+                                    const int e = e0 + lane, kr = e >> 3, c4 = e & 7;
+                                    const int64_t pk = __shfl_sync(0xffffffffu, pi, kr);
                                     if (pk >= 0)
-                                        reinterpret_cast<float4*>(a.part_o + pk * D)[c4] =
+                                        reinterpret_cast<float4*>(a.part_o + pk * D + c0)[c4] =
                                             *reinterpret_cast<const float4*>(ostage + kr * OSTR + c4 * 16);
                                 }
                                 __syncwarp();
@@ -677,51 +698,53 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         const int64_t deep0 = deep_row(s, a.layer, G.seq, h, G.A);  // first window row of plane R
         int iu = split + a.nsplit * ww;  // this warp's units: iu, iu + ustep, ...
         if (iu < nunits) {
-            // Copies of tile t of unit w into stage `stage`: 16-byte vectors in row
-            // order (a warp instruction covers 512 contiguous bytes of window rows);
+            // Copies of tile t of unit w into stage `stage`: a lane quad per row, 64
+            // contiguous bytes per quad and instruction (eight rows per instruction);
             // keys outside the window or past the unit's keys are zero-filled.
             auto issue = [&](const WinUnit& w, int t, int stage) {
                 uint8_t* sb = wbuf + stage * Lay::WSTAGE;
                 const bool ring = w.depth < s.R;
                 const int64_t wbase =
                     ring ? ring0 + (int64_t)(w.depth - 1) * plane_bytes + (int64_t)w.lo * 2 * D : deep0;
-                const char* kw = (ring ? s.kwin : s.kdeep) + wbase;
-                const char* vw = (ring ? s.vwin : s.vdeep) + wbase;
+                const int q4 = lane & 3, r8 = lane >> 2;
 #pragma unroll
-                for (int e0 = 0; e0 < kWinKeys * NV; e0 += 32) {
-                    const int e = e0 + lane, kr = e / NV, v = e - kr * NV;
+                for (int half = 0; half < 2; ++half) {
+                    const int kr = half * 8 + r8;
                     const int key = t * kWinKeys + kr;
                     const char* kp = a.Q;
                     const char* vp = a.Q;
                     bool ok;
                     if (key < w.wk) {
                         ok = win_valid(w, wkeys, s.R, s.Wcap, key);
+                        const int64_t off = wbase + (int64_t)key * 2 * D + q4 * 16;
                         if (ok) {
-                            kp = kw + (int64_t)key * 2 * D + v * 16;
-                            vp = vw + (int64_t)key * 2 * D + v * 16;
+                            kp = (ring ? s.kwin : s.kdeep) + off;
+                            vp = (ring ? s.vwin : s.vdeep) + off;
                         }
                     } else {
                         ok = key < w.nk;
                         if (ok) {
                             const int64_t off =
-                                (((int64_t)w.row0 + (int64_t)(key - w.wk) * w.stride) * s.H + h) * 2 * D + v * 16;
+                                (((int64_t)w.row0 + (int64_t)(key - w.wk) * w.stride) * s.H + h) * 2 * D + q4 * 16;
                             kp = a.Kb + off;
                             vp = a.Vb + off;
                         }
                     }
-                    cp_async16_zfill(sb + kr * WSTR + v * 16, kp, ok);
-                    cp_async16_zfill(sb + (kWinKeys + kr) * WSTR + v * 16, vp, ok);
+                    uint8_t* dk = sb + kr * WSTR + q4 * 16;
+#pragma unroll
+                    for (int j = 0; j < NV / 4; ++j) {
+                        cp_async16_zfill(dk + 64 * j, kp + (ok ? 64 * j : 0), ok);
+                        cp_async16_zfill(dk + kWinKeys * WSTR + 64 * j, vp + (ok ? 64 * j : 0), ok);
+                    }
                 }
                 if (t == 0) {
+                    const bool okq = r8 < w.nr;
+                    const char* qp = okq ? a.Q + (((int64_t)w.row0 + (int64_t)(w.j0 + r8) * w.stride) * s.H + h) *
+                                                     (2 * D) + q4 * 16
+                                         : a.Q;
+                    uint8_t* dq = sb + (2 * kWinKeys + r8) * WSTR + q4 * 16;
 #pragma unroll
-                    for (int e0 = 0; e0 < kWinRows * NV; e0 += 32) {
-                        const int e = e0 + lane, r = e / NV, v = e - r * NV;
-                        const bool okq = r < w.nr;
-                        const char* qp = okq ? a.Q + (((int64_t)w.row0 + (int64_t)(w.j0 + r) * w.stride) * s.H + h) *
-                                                         (2 * D) + v * 16
-                                             : a.Q;
-                        cp_async16_zfill(sb + (2 * kWinKeys + r) * WSTR + v * 16, qp, okq);
-                    }
+                    for (int j = 0; j < NV / 4; ++j) cp_async16_zfill(dq + 64 * j, qp + (okq ? 64 * j : 0), okq);
                 }
                 cp_async_commit();
             };
@@ -778,14 +801,16 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     m_a = m_b = -INFINITY;
                     l_a = l_b = 0.f;
                 }
-                // ---- S^T = K Q^T for 16 keys x 8 rows
-                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                // ---- S^T = K Q^T for 16 keys x 8 rows (two accumulation chains)
+                float c[4] = {0.f, 0.f, 0.f, 0.f}, c_odd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < NKS; ++ks) {
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4(sb + k_lane + 32 * ks, a0, a1, a2, a3);
-                    mma_16816(c, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+                    mma_16816((ks & 1) ? c_odd : c, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c[e] += c_odd[e];
                 // ---- visibility: window keys for every row, block token j' for rows j >= j'
                 const int k0 = ct * kWinKeys + (lane >> 2), k1 = k0 + 8;
                 const bool w0 = k0 < wc.wk && win_valid(wc, wkeys, s.R, s.Wcap, k0);
@@ -879,15 +904,31 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     if (G.nrows > 0 && !*abort_flag) {
         const int np = deep_splits_used(G.A, a.chunk, a.nsplit);
         const int sub = lane >> 3, sl = lane & 7;
-        for (int k = warp * 4; split + a.nsplit * k < G.nrows; k += NWARPS * 4) {
-            const int rl = split + a.nsplit * (k + sub);
-            const int row = rl < G.nrows ? group_row(bt, G.nb, rl) : -1;
-            if (row < 0) continue;
-            const int64_t ro = (int64_t)row * s.H + h;
-            if (np < 4)
-                merge_row<D, 4>(a, ro, np, sl);
-            else
-                merge_row_any<D>(a, ro, np, sl);
+        for (int k = warp * 8; split + a.nsplit * k < G.nrows; k += NWARPS * 8) {
+            int64_t ro[2];
+            bool ok[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int rl = split + a.nsplit * (k + sub + 4 * x);
+                const int row = group_row(rowtab, bt, G.nb, G.nrows, rl);
+                ok[x] = row >= 0;
+                ro[x] = ok[x] ? (int64_t)row * s.H + h : 0;
+            }
+            if (np < 3 && D <= 96) {
+                merge_rows<D, 3, 2>(a, ro, ok, np, sl);
+            } else if (np < 3) {
+                merge_rows<D, 3, 1>(a, ro, ok, np, sl);
+                merge_rows<D, 3, 1>(a, ro + 1, ok + 1, np, sl);
+            } else {
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (!ok[x]) continue;
+                    if (np < 4)
+                        merge_rows<D, 4, 1>(a, ro + x, ok + x, np, sl);
+                    else
+                        merge_row_any<D>(a.part_ml, a.part_o, a.O, a.lse, a.nseg, a.nsplit, ro[x], np, sl);
+                }
+            }
         }
     }
 }

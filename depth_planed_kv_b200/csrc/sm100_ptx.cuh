@@ -81,16 +81,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 // 16-byte asynchronous copy global -> shared, cached in L2 only (commit/wait groups).
+// No memory clobber: the destination is read only after cp_async_wait_*, which
+// carries one, so ordinary loads and arithmetic may be scheduled around the issue.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
-                 "l"(reinterpret_cast<uint64_t>(src))
-                 : "memory");
+                 "l"(reinterpret_cast<uint64_t>(src)));
 }
 // The same with a source size: `valid` false writes 16 zero bytes and reads nothing.
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(valid ? 16 : 0)
-                 : "memory");
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(valid ? 16 : 0));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -221,10 +221,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
-// C[16x8] += A[16x16] (row) * B[16x8] (col), bf16 inputs, fp32 accumulate.
+// C[16x8] += A[16x16] (row) * B[16x8] (col), bf16 inputs, fp32 accumulate.  Registers
+// only (not volatile): the compiler may interleave independent tiles.
 __device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                           uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -233,7 +234,7 @@ __device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, ui
 // Transpose an 8x8 matrix of 16-bit values held as one fragment register per lane.
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
     return y;
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
