@@ -34,7 +34,7 @@
 // 512-byte atoms): Q, K K-major in 32-element column chunks of [rows][64 B];
 // V MN-major (the same chunks read with head-dim as N); P K-major [128][32 keys]
 // chunks written by the softmax threads.  Window stages hold [16 K rows][16 V
-// rows][8 Q rows] at a padded stride of 2*d+16 bytes (conflict-free ldmatrix).
+// rows] at a padded stride of 2*d+16 bytes (conflict-free ldmatrix).
 #include <cuda.h>
 
 #include "ripe_launch.h"
@@ -67,7 +67,7 @@ struct FusedLayout {
     static constexpr int KV_STAGE = NCH * 4096;      // 64 keys x 64 B per chunk
     static constexpr int P_BUF = 2 * 8192;           // one M tile: 2 chunks of 32 keys
     static constexpr int WSTR = 2 * D + 16;          // window row stride (bytes)
-    static constexpr int WSTAGE = (2 * kWinKeys + kWinRows) * WSTR;
+    static constexpr int WSTAGE = 2 * kWinKeys * WSTR;  // K rows, then V rows
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
@@ -696,17 +696,33 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         const int64_t ring0 = ring_row(s, a.layer, G.seq, h, 1, 0);  // plane 1, slot 0
         const int64_t plane_bytes = (int64_t)s.Wcap * 2 * D;        // one ring plane
         const int64_t deep0 = deep_row(s, a.layer, G.seq, h, G.A);  // first window row of plane R
+        const int q4 = lane & 3, r8 = lane >> 2;
         int iu = split + a.nsplit * ww;  // this warp's units: iu, iu + ustep, ...
         if (iu < nunits) {
+            // Q^T fragments (B operand) of unit w straight from global memory:
+            // b0 = Q[j0 + lane/4][16 ks + 2 q4 ..], b1 the same 8 channels on; rows past nr are 0.
+            auto load_q = [&](const WinUnit& w, uint32_t (&b)[NKS][2]) {
+                const bool okq = r8 < w.nr;
+                const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+                    a.Q + (okq ? (((int64_t)w.row0 + (int64_t)(w.j0 + r8) * w.stride) * s.H + h) * (2 * D) : 0));
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    b[ks][0] = okq ? __ldg(qp + 8 * ks + q4) : 0u;
+                    b[ks][1] = okq ? __ldg(qp + 8 * ks + 4 + q4) : 0u;
+                }
+            };
+            // Window rows of unit w start here (ring plane slot lo, or plane R row A).
+            auto win_base = [&](const WinUnit& w, const char*& kw, const char*& vw) {
+                const bool ring = w.depth < s.R;
+                const int64_t wb = ring ? ring0 + (int64_t)(w.depth - 1) * plane_bytes + (int64_t)w.lo * 2 * D : deep0;
+                kw = (ring ? s.kwin : s.kdeep) + wb;
+                vw = (ring ? s.vwin : s.vdeep) + wb;
+            };
             // Copies of tile t of unit w into stage `stage`: a lane quad per row, 64
             // contiguous bytes per quad and instruction (eight rows per instruction);
             // keys outside the window or past the unit's keys are zero-filled.
-            auto issue = [&](const WinUnit& w, int t, int stage) {
+            auto issue = [&](const WinUnit& w, const char* kw, const char* vw, int t, int stage) {
                 uint8_t* sb = wbuf + stage * Lay::WSTAGE;
-                const bool ring = w.depth < s.R;
-                const int64_t wbase =
-                    ring ? ring0 + (int64_t)(w.depth - 1) * plane_bytes + (int64_t)w.lo * 2 * D : deep0;
-                const int q4 = lane & 3, r8 = lane >> 2;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const int kr = half * 8 + r8;
@@ -716,10 +732,9 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     bool ok;
                     if (key < w.wk) {
                         ok = win_valid(w, wkeys, s.R, s.Wcap, key);
-                        const int64_t off = wbase + (int64_t)key * 2 * D + q4 * 16;
                         if (ok) {
-                            kp = (ring ? s.kwin : s.kdeep) + off;
-                            vp = (ring ? s.vwin : s.vdeep) + off;
+                            kp = kw + key * (2 * D) + q4 * 16;
+                            vp = vw + key * (2 * D) + q4 * 16;
                         }
                     } else {
                         ok = key < w.nk;
@@ -737,119 +752,137 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         cp_async16_zfill(dk + kWinKeys * WSTR + 64 * j, vp + (ok ? 64 * j : 0), ok);
                     }
                 }
-                if (t == 0) {
-                    const bool okq = r8 < w.nr;
-                    const char* qp = okq ? a.Q + (((int64_t)w.row0 + (int64_t)(w.j0 + r8) * w.stride) * s.H + h) *
-                                                     (2 * D) + q4 * 16
-                                         : a.Q;
-                    uint8_t* dq = sb + (2 * kWinKeys + r8) * WSTR + q4 * 16;
-#pragma unroll
-                    for (int j = 0; j < NV / 4; ++j) cp_async16_zfill(dq + 64 * j, qp + (okq ? 64 * j : 0), okq);
-                }
                 cp_async_commit();
             };
 
             WinUnit wi = win_unit(bt, G.nb, iu, wkeys, s.R, lane);
             WinUnit wc = wi;
+            const char *kwi, *vwi;
+            win_base(wi, kwi, vwi);
             int cu = iu, it_ = 0, ct = 0;
             bool ihas = true;
             auto advance_issue = [&]() {
                 if (++it_ == wi.ntiles) {
                     iu += ustep;
                     it_ = 0;
-                    if (iu < nunits)
+                    if (iu < nunits) {
                         wi = win_unit(bt, G.nb, iu, wkeys, s.R, lane);
-                    else
+                        win_base(wi, kwi, vwi);
+                    } else {
                         ihas = false;
+                    }
                 }
             };
 #pragma unroll
             for (int sidx = 0; sidx < NS - 1; ++sidx) {
                 if (ihas) {
-                    issue(wi, it_, sidx);
+                    issue(wi, kwi, vwi, it_, sidx);
                     advance_issue();
                 } else {
                     cp_async_commit();
                 }
             }
 
-            uint32_t bq[NKS][2];
+            uint32_t bq[NKS][2], bq_next[NKS][2];
+            load_q(wc, bq_next);
             float o[NMT][4];
             float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-            const int ra = 2 * (lane & 3), rb = ra + 1;  // fragment columns (rows) of this lane
+            const int ra = 2 * q4, rb = ra + 1;  // fragment columns (rows) of this lane
             const uint32_t k_lane = ((lane & 7) + 8 * ((lane >> 3) & 1)) * WSTR + 16 * (lane >> 4);
             const uint32_t v_lane = kWinKeys * WSTR + ((lane & 7) + 8 * (lane >> 4)) * WSTR + 16 * ((lane >> 3) & 1);
-            const uint32_t q_lane = 2 * kWinKeys * WSTR + (lane & 7) * WSTR + 16 * (lane >> 3);
             for (int q = 0;; ++q) {
                 if (ihas) {
-                    issue(wi, it_, (q + NS - 1) % NS);
+                    issue(wi, kwi, vwi, it_, (q + NS - 1) % NS);
                     advance_issue();
                 } else {
                     cp_async_commit();
                 }
-                cp_async_wait_group<NS - 1>();
-                __syncwarp();
-                const uint32_t sb = wbuf_a + (q % NS) * Lay::WSTAGE;
                 if (ct == 0) {
-                    // Q^T fragments (B operand, k-steps in pairs) and a fresh accumulator.
+                    // A new unit: its Q^T fragments (loaded one unit ahead), the next unit's
+                    // fragments in flight, a fresh accumulator.
 #pragma unroll
-                    for (int s2 = 0; s2 < NKS / 2; ++s2)
-                        ldsm_x4(sb + q_lane + 64 * s2, bq[2 * s2][0], bq[2 * s2][1], bq[2 * s2 + 1][0],
-                                bq[2 * s2 + 1][1]);
+                    for (int ks = 0; ks < NKS; ++ks) {
+                        bq[ks][0] = bq_next[ks][0];
+                        bq[ks][1] = bq_next[ks][1];
+                    }
+                    if (cu + ustep < nunits) load_q(win_unit(bt, G.nb, cu + ustep, wkeys, s.R, lane), bq_next);
 #pragma unroll
                     for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
                     m_a = m_b = -INFINITY;
                     l_a = l_b = 0.f;
                 }
+                cp_async_wait_group<NS - 1>();
+                __syncwarp();
+                const uint32_t sb = smem_ready(wbuf_a + (q % NS) * Lay::WSTAGE);
                 // ---- S^T = K Q^T for 16 keys x 8 rows (two accumulation chains)
                 float c[4] = {0.f, 0.f, 0.f, 0.f}, c_odd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < NKS; ++ks) {
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4(sb + k_lane + 32 * ks, a0, a1, a2, a3);
+                    ldsm_x4_r(sb + k_lane + 32 * ks, a0, a1, a2, a3);
                     mma_16816((ks & 1) ? c_odd : c, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) c[e] += c_odd[e];
-                // ---- visibility: window keys for every row, block token j' for rows j >= j'
+                float s0 = (c[0] + c_odd[0]) * c2, s1 = (c[1] + c_odd[1]) * c2;
+                float s2 = (c[2] + c_odd[2]) * c2, s3 = (c[3] + c_odd[3]) * c2;
+                // ---- visibility: window slots inside the window for every row, block
+                // token j' for rows j >= j'.  Rows past nr are never written: unmasked.
                 const int k0 = ct * kWinKeys + (lane >> 2), k1 = k0 + 8;
                 const bool w0 = k0 < wc.wk && win_valid(wc, wkeys, s.R, s.Wcap, k0);
                 const bool w1 = k1 < wc.wk && win_valid(wc, wkeys, s.R, s.Wcap, k1);
-                auto vis = [&](int key, bool win, int r) {
-                    return r < wc.nr && key < wc.nk && (key < wc.wk ? win : key - wc.wk <= wc.j0 + r);
-                };
-                const float s0 = vis(k0, w0, ra) ? c[0] * c2 : -INFINITY;
-                const float s1 = vis(k0, w0, rb) ? c[1] * c2 : -INFINITY;
-                const float s2 = vis(k1, w1, ra) ? c[2] * c2 : -INFINITY;
-                const float s3 = vis(k1, w1, rb) ? c[3] * c2 : -INFINITY;
-                float mx_a = fmaxf(s0, s2), mx_b = fmaxf(s1, s3);
-#pragma unroll
-                for (int o2 = 4; o2 < 32; o2 <<= 1) {
-                    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, o2));
-                    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, o2));
+                if (!__all_sync(0xffffffffu, w0 && w1)) {
+                    const int jr_a = wc.j0 + ra + wc.wk, jr_b = jr_a + 1;  // last visible key of rows ra, rb
+                    const bool v0 = k0 < wc.wk ? w0 : k0 < wc.nk;
+                    const bool v1 = k1 < wc.wk ? w1 : k1 < wc.nk;
+                    if (!(v0 && (k0 < wc.wk || k0 <= jr_a))) s0 = -INFINITY;
+                    if (!(v0 && (k0 < wc.wk || k0 <= jr_b))) s1 = -INFINITY;
+                    if (!(v1 && (k1 < wc.wk || k1 <= jr_a))) s2 = -INFINITY;
+                    if (!(v1 && (k1 < wc.wk || k1 <= jr_b))) s3 = -INFINITY;
                 }
-                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-                const float al_a = mn_a == -INFINITY ? 1.f : ex2(m_a - mn_a);
-                const float al_b = mn_b == -INFINITY ? 1.f : ex2(m_b - mn_b);
-                const float p0 = mn_a == -INFINITY ? 0.f : ex2(s0 - mn_a);
-                const float p1 = mn_b == -INFINITY ? 0.f : ex2(s1 - mn_b);
-                const float p2 = mn_a == -INFINITY ? 0.f : ex2(s2 - mn_a);
-                const float p3 = mn_b == -INFINITY ? 0.f : ex2(s3 - mn_b);
-                l_a = l_a * al_a + (p0 + p2);
-                l_b = l_b * al_b + (p1 + p3);
-                m_a = mn_a;
-                m_b = mn_b;
+                // The running max m of a row moves only when a score exceeds it by more
+                // than 2^8 (probabilities then stay below 256).  Only then is the tile's
+                // row max reduced across the lanes; lanes of a row decide alike.
+                const bool over = fmaxf(s0, s2) > m_a + 8.f || fmaxf(s1, s3) > m_b + 8.f;
+                if (__any_sync(0xffffffffu, over)) {
+                    float mx_a = fmaxf(s0, s2), mx_b = fmaxf(s1, s3);
+#pragma unroll
+                    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, o2));
+                        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, o2));
+                    }
+                    if (mx_a > m_a + 8.f) {
+                        const float al = ex2(m_a - mx_a);
+                        m_a = mx_a;
+                        l_a *= al;
+#pragma unroll
+                        for (int mt = 0; mt < NMT; ++mt) {
+                            o[mt][0] *= al;
+                            o[mt][2] *= al;
+                        }
+                    }
+                    if (mx_b > m_b + 8.f) {
+                        const float al = ex2(m_b - mx_b);
+                        m_b = mx_b;
+                        l_b *= al;
+#pragma unroll
+                        for (int mt = 0; mt < NMT; ++mt) {
+                            o[mt][1] *= al;
+                            o[mt][3] *= al;
+                        }
+                    }
+                }
+                const float p0 = m_a == -INFINITY ? 0.f : ex2(s0 - m_a);
+                const float p1 = m_b == -INFINITY ? 0.f : ex2(s1 - m_b);
+                const float p2 = m_a == -INFINITY ? 0.f : ex2(s2 - m_a);
+                const float p3 = m_b == -INFINITY ? 0.f : ex2(s3 - m_b);
+                l_a += p0 + p2;
+                l_b += p1 + p3;
                 // ---- O^T += V^T P^T: P^T by an 8x8 transpose of the S^T fragments
                 const uint32_t b0 = movmatrix_t(pack_bf16(p0, p1));
                 const uint32_t b1 = movmatrix_t(pack_bf16(p2, p3));
 #pragma unroll
                 for (int mt = 0; mt < NMT; ++mt) {
-                    o[mt][0] *= al_a;
-                    o[mt][1] *= al_b;
-                    o[mt][2] *= al_a;
-                    o[mt][3] *= al_b;
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(sb + v_lane + 32 * mt, a0, a1, a2, a3);
+                    ldsm_x4_t_r(sb + v_lane + 32 * mt, a0, a1, a2, a3);
                     mma_16816(o[mt], a0, a1, a2, a3, b0, b1);
                 }
                 if (ct == wc.ntiles - 1) {
@@ -985,12 +1018,12 @@ cudaError_t launch_fused(const void* tmK, const void* tmV, const VerifyArgs& a, 
     const int d = a.s.d;
     // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
     if (mt == 1) {
-        if (d == 64) return launch_t<64, 1, 4, 4, 3>(tk, tv, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 1, 2, 4, 3>(tk, tv, a, gslots, pdl, st);
-        if (d == 128) return launch_t<128, 1, 2, 4, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 64) return launch_t<64, 1, 4, 6, 3>(tk, tv, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 1, 3, 6, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 1, 2, 5, 2>(tk, tv, a, gslots, pdl, st);
     } else {
-        if (d == 64) return launch_t<64, 2, 3, 4, 3>(tk, tv, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 2, 2, 3, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 64) return launch_t<64, 2, 3, 6, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 2, 2, 4, 2>(tk, tv, a, gslots, pdl, st);
         if (d == 128) return launch_t<128, 2, 2, 1, 2>(tk, tv, a, gslots, pdl, st);
     }
     return cudaErrorInvalidValue;

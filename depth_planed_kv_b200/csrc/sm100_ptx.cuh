@@ -221,6 +221,24 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
+// The same loads as plain (reorderable) asm, for callers that make the address
+// depend on a point after which the shared memory is ready (see smem_ready).
+__device__ __forceinline__ void ldsm_x4_r(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+        : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t_r(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+        : "r"(addr));
+}
+// Returns `addr` through an opaque step placed here in program order: loads whose
+// address derives from the result cannot be hoisted above this point.
+__device__ __forceinline__ uint32_t smem_ready(uint32_t addr) {
+    asm volatile("" : "+r"(addr)::"memory");
+    return addr;
+}
 // C[16x8] += A[16x16] (row) * B[16x8] (col), bf16 inputs, fp32 accumulate.  Registers
 // only (not volatile): the compiler may interleave independent tiles.
 __device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
