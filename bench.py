@@ -37,7 +37,7 @@ from depth_planed_kv_b200 import synth as S  # noqa: E402
 METRIC = "RIPE verify-attn KV GB/s + query-rows/s (1×B200), % of HBM roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM = 6650.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PROFILES_DIR = os.path.join(ROOT, "profiles")
 
 
 def algorithmic_bytes(wl, T, ws, branches, with_lse=True):
@@ -84,15 +84,28 @@ def kernel_source_hash():
 
 
 def traffic_for(workload: str):
-    """ncu DRAM bytes per launch of the dominant kernel, if captured on the current source."""
+    """ncu DRAM bytes (read + write) per launch of the dominant kernel, if a summary
+    under profiles/ records them for this workload on the current kernel source.
+
+    A summary carries one line of the form
+    ``traffic: workload=<name> source_hash=<hash> dram_bytes_per_launch=<int>``.
+    """
+    want = kernel_source_hash()
     try:
-        with open(TRAFFIC_FILE) as f:
-            t = json.load(f)
-        e = t.get(workload)
-        if e and e.get("source_hash") == kernel_source_hash():
-            return e.get("dram_bytes_per_launch")
-    except Exception:
-        pass
+        names = sorted(os.listdir(PROFILES_DIR))
+    except OSError:
+        return None
+    for name in names:
+        if not name.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(PROFILES_DIR, name)) as f:
+            for line in f:
+                line = line.strip().strip("`")
+                if not line.startswith("traffic:"):
+                    continue
+                kv = dict(x.split("=", 1) for x in line[len("traffic:"):].split() if "=" in x)
+                if kv.get("workload") == workload and kv.get("source_hash") == want:
+                    return int(kv["dram_bytes_per_launch"])
     return None
 
 
