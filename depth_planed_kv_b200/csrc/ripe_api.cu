@@ -203,7 +203,7 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
     c->kwin = c->base + y.kwin; c->vwin = c->base + y.vwin;
     c->len = (int32_t*)(c->base + y.len); c->ws = (int32_t*)(c->base + y.ws);
     c->err = (int32_t*)(c->base + y.err);
-    c->tc_ready = fused_supported(dtype, d) && make_deep_tensor_maps(c) == 0;
+    c->tc_ready = fused_supported(dtype, d) && make_tensor_maps(c) == 0;
     // Zeroed store: key tiles that overrun a region read finite values.
     cudaError_t e = cudaMemset(c->base, 0, y.total);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();

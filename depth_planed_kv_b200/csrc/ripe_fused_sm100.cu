@@ -33,8 +33,8 @@
 // Shared-memory operand layouts of the deep part (64-byte swizzle, 8-row /
 // 512-byte atoms): Q, K K-major in 32-element column chunks of [rows][64 B];
 // V MN-major (the same chunks read with head-dim as N); P K-major [128][32 keys]
-// chunks written by the softmax threads.  Window stages hold [16 K rows][16 V
-// rows] at a padded stride of 2*d+16 bytes (conflict-free ldmatrix).
+// chunks written by the softmax threads.  Window stages hold the K and V rows of
+// 16 keys in the same 64-byte-swizzled 32-column boxes (conflict-free ldmatrix).
 #include <cuda.h>
 
 #include "ripe_launch.h"
@@ -49,6 +49,12 @@ constexpr int kMaxGroupBranches = 64;
 constexpr int kWinRows = 8;   // rows per window unit (the N of an m16n8k16 tile)
 constexpr int kWinKeys = 16;  // keys per window tile (the M of an m16n8k16 tile)
 constexpr int kRowTable = 512;  // group rows whose Q/O row index is tabulated in shared memory
+
+// Tensor maps of one launch: deep K, V in 64-row boxes; ring K, V and deep K, V
+// in 16-row boxes (all 32 columns wide, 64-byte swizzle).
+struct TMaps {
+    CUtensorMap dk, dv, wk, wv, rk, rv;
+};
 
 // One branch of the group: its rows, its offset among the group's rows, its
 // depth and the index of its first window unit.
@@ -66,8 +72,9 @@ struct FusedLayout {
     static constexpr int Q_BYTES = MT * NCH * 8192;  // 128 rows x 64 B per chunk
     static constexpr int KV_STAGE = NCH * 4096;      // 64 keys x 64 B per chunk
     static constexpr int P_BUF = 2 * 8192;           // one M tile: 2 chunks of 32 keys
-    static constexpr int WSTR = 2 * D + 16;          // window row stride (bytes)
-    static constexpr int WSTAGE = 2 * kWinKeys * WSTR;  // K rows, then V rows
+    static constexpr int WBOX = kWinKeys * 64;       // one 16-row x 64-byte window box
+    static constexpr int WKV = NCH * WBOX;           // K (or V) of one window tile
+    static constexpr int WSTAGE = 2 * WKV;           // K boxes, then V boxes
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
@@ -76,7 +83,8 @@ struct FusedLayout {
     static constexpr int OFF_BAR = OFF_W + NW * NS * WSTAGE;
     // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
     static constexpr int NBAR = 1 + 3 * ST + 7;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;  // one per window stage
+    static constexpr int OFF_MISC = OFF_WBAR + NW * NS * 8;
     static constexpr int OFF_BT = OFF_MISC + 64;
     static constexpr int OFF_RT = OFF_BT + kMaxGroupBranches * (int)sizeof(BranchEnt);
     static constexpr int BYTES = OFF_RT + kRowTable * 4;
@@ -227,6 +235,7 @@ __device__ __forceinline__ void merge_rows(const VerifyArgs& a, const int64_t* r
             }
         }
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro[r] * D;
+        const float inv = 1.f / L;
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -240,7 +249,7 @@ __device__ __forceinline__ void merge_rows(const VerifyArgs& a, const int64_t* r
                 }
             }
             *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
-                make_uint2(pack_bf16(acc[0] / L, acc[1] / L), pack_bf16(acc[2] / L, acc[3] / L));
+                make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
         }
         if (sl == 0 && a.lse) a.lse[ro[r]] = (M + log2f(L)) * 0.69314718055994531f;
     }
@@ -275,10 +284,11 @@ __device__ __noinline__ void merge_row_any(const float2* part_ml, const float* p
         }
     }
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(O_) + ro * D;
+    const float inv = 1.f / L;
 #pragma unroll
     for (int c = 0; c < CH; ++c)
         *reinterpret_cast<uint2*>(orow + 4 * sl + 32 * c) =
-            make_uint2(pack_bf16(acc[c][0] / L, acc[c][1] / L), pack_bf16(acc[c][2] / L, acc[c][3] / L));
+            make_uint2(pack_bf16(acc[c][0] * inv, acc[c][1] * inv), pack_bf16(acc[c][2] * inv, acc[c][3] * inv));
     if (sl == 0 && lse) lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
 }
 
@@ -286,7 +296,7 @@ __device__ __noinline__ void merge_row_any(const float2* part_ml, const float* p
 // which hold ceil(warps / 4) warps apiece: 168 per thread for 9-12 warps.
 template <int D, int MT, int ST, int NW, int NS>
 __global__ void __launch_bounds__(FusedLayout<D, MT, ST, NW, NS>::THREADS, 1)
-verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, VerifyArgs a) {
+verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
     using Lay = FusedLayout<D, MT, ST, NW, NS>;
     using namespace sm100;
     constexpr int NCH = Lay::NCH;
@@ -333,6 +343,7 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             mbar_init(pv_done + i, 1);
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < NW * NS; ++i) mbar_init(reinterpret_cast<uint64_t*>(sm + Lay::OFF_WBAR) + i, 32);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -341,8 +352,8 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         tmem_relinquish();
     }
     if (warp == 4 && lane == 0) {
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
+        prefetch_tmap(&tm.dk);
+        prefetch_tmap(&tm.dv);
     }
     tc_fence_before();
     __syncthreads();
@@ -435,11 +446,11 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         mbar_expect_tx(k_full + st, Lay::KV_STAGE);
 #pragma unroll
                         for (int c = 0; c < NCH; ++c)
-                            tma_load_2d(sK + st * Lay::KV_STAGE + c * 4096, &tmK, 32 * c, y, k_full + st);
+                            tma_load_2d(sK + st * Lay::KV_STAGE + c * 4096, &tm.dk, 32 * c, y, k_full + st);
                         mbar_expect_tx(v_full + st, Lay::KV_STAGE);
 #pragma unroll
                         for (int c = 0; c < NCH; ++c)
-                            tma_load_2d(sV + st * Lay::KV_STAGE + c * 4096, &tmV, 32 * c, y, v_full + st);
+                            tma_load_2d(sV + st * Lay::KV_STAGE + c * 4096, &tm.dv, 32 * c, y, v_full + st);
                     }
                     if (*abort_flag) {
                         // Let the copies already issued land before the CTA's shared memory goes away.
@@ -531,7 +542,7 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                             const int row = group_row(rowtab, bt, G.nb, G.nrows, rt * RT + mt * 128 + t);
                             rows[mt] = row;
                             constexpr int QV = 2 * D / 16;  // 16-byte vectors per row
-#pragma unroll
+#pragma unroll 1
                             for (int e0 = 0; e0 < 32 * QV; e0 += 32) {
                                 const int e = e0 + lane, r = e / QV, v = e - r * QV;
                                 const int rrow = __shfl_sync(0xffffffffu, row, r);
@@ -621,7 +632,7 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                                 break;
                             }
                             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                             for (int c0 = 0; c0 < D; c0 += 32) {
                                 float o[32];
                                 tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
@@ -682,21 +693,25 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         }
     } else if (G.units > 0) {
         // ------------------------------------------------ window warps
-        constexpr int WSTR = Lay::WSTR;
-        constexpr int NV = 2 * D / 16;  // 16-byte vectors per row
-        constexpr int NKS = D / 16;     // k-steps of S^T = K Q^T
-        constexpr int NMT = D / 16;     // 16-channel tiles of O^T
+        constexpr int NKS = D / 16;  // k-steps of S^T = K Q^T
+        constexpr int NMT = D / 16;  // 16-channel tiles of O^T
         const int ww = warp - 6;
         uint8_t* wbuf = sm + Lay::OFF_W + ww * NS * Lay::WSTAGE;
+        uint64_t* wbar = reinterpret_cast<uint64_t*>(sm + Lay::OFF_WBAR) + ww * NS;
         const uint32_t wbuf_a = smem_u32(wbuf);
         const WinKeys wkeys = win_keys(G.A, G.T, s.Wcap);
         const int ustep = a.nsplit * NW;
         const int nunits = G.units;
         const float c2 = a.scale_log2;
-        const int64_t ring0 = ring_row(s, a.layer, G.seq, h, 1, 0);  // plane 1, slot 0
-        const int64_t plane_bytes = (int64_t)s.Wcap * 2 * D;        // one ring plane
-        const int64_t deep0 = deep_row(s, a.layer, G.seq, h, G.A);  // first window row of plane R
+        // Row indices, in the 2-D tensor-map views, of ring plane 1 slot 0 and of the
+        // first window row of plane R.
+        const int ring_y0 = ((a.layer * s.Bmax + G.seq) * s.H + h) * (s.R - 1) * s.Wcap;
+        const int deep_y0 = ((a.layer * s.Bmax + G.seq) * s.H + h) * s.Tmax + G.A;
         const int q4 = lane & 3, r8 = lane >> 2;
+        if (lane == 0) {
+            prefetch_tmap(&tm.wk);
+            prefetch_tmap(&tm.wv);
+        }
         int iu = split + a.nsplit * ww;  // this warp's units: iu, iu + ustep, ...
         if (iu < nunits) {
             // Q^T fragments (B operand) of unit w straight from global memory:
@@ -711,30 +726,48 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     b[ks][1] = okq ? __ldg(qp + 8 * ks + 4 + q4) : 0u;
                 }
             };
-            // Window rows of unit w start here (ring plane slot lo, or plane R row A).
-            auto win_base = [&](const WinUnit& w, const char*& kw, const char*& vw) {
-                const bool ring = w.depth < s.R;
-                const int64_t wb = ring ? ring0 + (int64_t)(w.depth - 1) * plane_bytes + (int64_t)w.lo * 2 * D : deep0;
-                kw = (ring ? s.kwin : s.kdeep) + wb;
-                vw = (ring ? s.vwin : s.vdeep) + wb;
-            };
-            // Copies of tile t of unit w into stage `stage`: a lane quad per row, 64
-            // contiguous bytes per quad and instruction (eight rows per instruction);
-            // keys outside the window or past the unit's keys are zero-filled.
-            auto issue = [&](const WinUnit& w, const char* kw, const char* vw, int t, int stage) {
+            // Tile t of unit w into stage `stage`, in the 64-byte-swizzled box layout
+            // (row r, 16-byte chunk c of column block b at b*WBOX + r*64 + ((c ^ (r>>1 & 3)) << 4)).
+            // Tiles of window keys only: one lane issues the TMA boxes.  Tiles that hold
+            // draft-block keys: lane quads copy rows (zero-filling keys outside the
+            // window or past the unit); each lane's arrival waits for its copies.
+            auto issue = [&](const WinUnit& w, int t, int stage) {
                 uint8_t* sb = wbuf + stage * Lay::WSTAGE;
+                uint64_t* bar = wbar + stage;
+                const bool ring = w.depth < s.R;
+                const int k0t = t * kWinKeys;
+                if (k0t + kWinKeys <= w.wk) {
+                    if (lane == 0) {
+                        const int y = (ring ? ring_y0 + (w.depth - 1) * s.Wcap + w.lo : deep_y0) + k0t;
+                        const CUtensorMap* mk = ring ? &tm.wk : &tm.rk;
+                        const CUtensorMap* mv = ring ? &tm.wv : &tm.rv;
+                        fence_proxy_async_smem();  // earlier reads of this stage come first
+                        mbar_expect_tx(bar, Lay::WSTAGE);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c) {
+                            tma_load_2d(sb + c * Lay::WBOX, mk, 32 * c, y, bar);
+                            tma_load_2d(sb + Lay::WKV + c * Lay::WBOX, mv, 32 * c, y, bar);
+                        }
+                    } else {
+                        mbar_arrive(bar);
+                    }
+                    return;
+                }
+                const int64_t wbase = ring ? ring_row(s, a.layer, G.seq, h, w.depth, w.lo)
+                                           : deep_row(s, a.layer, G.seq, h, G.A);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const int kr = half * 8 + r8;
-                    const int key = t * kWinKeys + kr;
+                    const int key = k0t + kr;
                     const char* kp = a.Q;
                     const char* vp = a.Q;
                     bool ok;
                     if (key < w.wk) {
                         ok = win_valid(w, wkeys, s.R, s.Wcap, key);
+                        const int64_t off = wbase + (int64_t)key * 2 * D + q4 * 16;
                         if (ok) {
-                            kp = kw + key * (2 * D) + q4 * 16;
-                            vp = vw + key * (2 * D) + q4 * 16;
+                            kp = (ring ? s.kwin : s.kdeep) + off;
+                            vp = (ring ? s.vwin : s.vdeep) + off;
                         }
                     } else {
                         ok = key < w.nk;
@@ -745,58 +778,54 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                             vp = a.Vb + off;
                         }
                     }
-                    uint8_t* dk = sb + kr * WSTR + q4 * 16;
+                    uint8_t* dk = sb + kr * 64 + ((q4 ^ ((kr >> 1) & 3)) << 4);
 #pragma unroll
-                    for (int j = 0; j < NV / 4; ++j) {
-                        cp_async16_zfill(dk + 64 * j, kp + (ok ? 64 * j : 0), ok);
-                        cp_async16_zfill(dk + kWinKeys * WSTR + 64 * j, vp + (ok ? 64 * j : 0), ok);
+                    for (int j = 0; j < NCH; ++j) {
+                        cp_async16_zfill(dk + j * Lay::WBOX, kp + (ok ? 64 * j : 0), ok);
+                        cp_async16_zfill(dk + Lay::WKV + j * Lay::WBOX, vp + (ok ? 64 * j : 0), ok);
                     }
                 }
-                cp_async_commit();
+                cp_async_mbar_arrive(bar);
             };
 
             WinUnit wi = win_unit(bt, G.nb, iu, wkeys, s.R, lane);
             WinUnit wc = wi;
-            const char *kwi, *vwi;
-            win_base(wi, kwi, vwi);
             int cu = iu, it_ = 0, ct = 0;
             bool ihas = true;
+            int issued = 0;  // tiles issued (stage q % NS holds tile q)
             auto advance_issue = [&]() {
                 if (++it_ == wi.ntiles) {
                     iu += ustep;
                     it_ = 0;
-                    if (iu < nunits) {
+                    if (iu < nunits)
                         wi = win_unit(bt, G.nb, iu, wkeys, s.R, lane);
-                        win_base(wi, kwi, vwi);
-                    } else {
+                    else
                         ihas = false;
-                    }
                 }
             };
-#pragma unroll
-            for (int sidx = 0; sidx < NS - 1; ++sidx) {
-                if (ihas) {
-                    issue(wi, kwi, vwi, it_, sidx);
-                    advance_issue();
-                } else {
-                    cp_async_commit();
-                }
-            }
 
             uint32_t bq[NKS][2], bq_next[NKS][2];
             load_q(wc, bq_next);
             float o[NMT][4];
             float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
             const int ra = 2 * q4, rb = ra + 1;  // fragment columns (rows) of this lane
-            const uint32_t k_lane = ((lane & 7) + 8 * ((lane >> 3) & 1)) * WSTR + 16 * (lane >> 4);
-            const uint32_t v_lane = kWinKeys * WSTR + ((lane & 7) + 8 * (lane >> 4)) * WSTR + 16 * ((lane >> 3) & 1);
-            for (int q = 0;; ++q) {
+            // ldmatrix row addresses in the swizzled layout: K (A operand, rows = keys)
+            // and V (A operand of O^T by .trans, rows = keys).
+            const int rk = (lane & 7) + 8 * ((lane >> 3) & 1), rv = (lane & 7) + 8 * (lane >> 4);
+            const uint32_t k_row = rk * 64, v_row = Lay::WKV + rv * 64;
+            const uint32_t k_sw0 = (((lane >> 4) + 0) ^ ((rk >> 1) & 3)) << 4;
+            const uint32_t k_sw1 = (((lane >> 4) + 2) ^ ((rk >> 1) & 3)) << 4;
+            const uint32_t v_sw0 = ((((lane >> 3) & 1) + 0) ^ ((rv >> 1) & 3)) << 4;
+            const uint32_t v_sw1 = ((((lane >> 3) & 1) + 2) ^ ((rv >> 1) & 3)) << 4;
+            bool wok = true;
+            // Iterations q < 0 only fill the first NS-1 stages (tile q+NS-1 into its stage).
+            for (int q = 1 - NS;; ++q) {
                 if (ihas) {
-                    issue(wi, kwi, vwi, it_, (q + NS - 1) % NS);
+                    issue(wi, it_, (q + NS - 1) % NS);
+                    ++issued;
                     advance_issue();
-                } else {
-                    cp_async_commit();
                 }
+                if (q < 0) continue;
                 if (ct == 0) {
                     // A new unit: its Q^T fragments (loaded one unit ahead), the next unit's
                     // fragments in flight, a fresh accumulator.
@@ -811,15 +840,17 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     m_a = m_b = -INFINITY;
                     l_a = l_b = 0.f;
                 }
-                cp_async_wait_group<NS - 1>();
-                __syncwarp();
+                if (!warp_wait(wbar + q % NS, (q / NS) & 1, abort_flag, s.err)) {
+                    wok = false;
+                    break;
+                }
                 const uint32_t sb = smem_ready(wbuf_a + (q % NS) * Lay::WSTAGE);
                 // ---- S^T = K Q^T for 16 keys x 8 rows (two accumulation chains)
                 float c[4] = {0.f, 0.f, 0.f, 0.f}, c_odd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < NKS; ++ks) {
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4_r(sb + k_lane + 32 * ks, a0, a1, a2, a3);
+                    ldsm_x4_r(sb + (ks >> 1) * Lay::WBOX + k_row + ((ks & 1) ? k_sw1 : k_sw0), a0, a1, a2, a3);
                     mma_16816((ks & 1) ? c_odd : c, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
                 }
                 float s0 = (c[0] + c_odd[0]) * c2, s1 = (c[1] + c_odd[1]) * c2;
@@ -882,7 +913,7 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
 #pragma unroll
                 for (int mt = 0; mt < NMT; ++mt) {
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t_r(sb + v_lane + 32 * mt, a0, a1, a2, a3);
+                    ldsm_x4_t_r(sb + (mt >> 1) * Lay::WBOX + v_row + ((mt & 1) ? v_sw1 : v_sw0), a0, a1, a2, a3);
                     mma_16816(o[mt], a0, a1, a2, a3, b0, b1);
                 }
                 if (ct == wc.ntiles - 1) {
@@ -922,6 +953,12 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     ct = 0;
                 }
             }
+            if (!wok) {
+                // Let every issued tile land before the CTA's shared memory goes away.
+                volatile int no_abort = 0;
+                for (int qq = issued > NS ? issued - NS : 0; qq < issued; ++qq)
+                    mbar_wait(wbar + qq % NS, (qq / NS) & 1, &no_abort, s.err);
+            }
             cp_async_wait_all();
         }
     }
@@ -937,38 +974,21 @@ verify_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     if (G.nrows > 0 && !*abort_flag) {
         const int np = deep_splits_used(G.A, a.chunk, a.nsplit);
         const int sub = lane >> 3, sl = lane & 7;
-        for (int k = warp * 8; split + a.nsplit * k < G.nrows; k += NWARPS * 8) {
-            int64_t ro[2];
-            bool ok[2];
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int rl = split + a.nsplit * (k + sub + 4 * x);
-                const int row = group_row(rowtab, bt, G.nb, G.nrows, rl);
-                ok[x] = row >= 0;
-                ro[x] = ok[x] ? (int64_t)row * s.H + h : 0;
-            }
-            if (np < 3 && D <= 96) {
-                merge_rows<D, 3, 2>(a, ro, ok, np, sl);
-            } else if (np < 3) {
-                merge_rows<D, 3, 1>(a, ro, ok, np, sl);
-                merge_rows<D, 3, 1>(a, ro + 1, ok + 1, np, sl);
-            } else {
-#pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    if (!ok[x]) continue;
-                    if (np < 4)
-                        merge_rows<D, 4, 1>(a, ro + x, ok + x, np, sl);
-                    else
-                        merge_row_any<D>(a.part_ml, a.part_o, a.O, a.lse, a.nseg, a.nsplit, ro[x], np, sl);
-                }
-            }
+        for (int k = warp * 4; split + a.nsplit * k < G.nrows; k += NWARPS * 4) {
+            const int rl = split + a.nsplit * (k + sub);
+            const int row = group_row(rowtab, bt, G.nb, G.nrows, rl);
+            const bool ok = row >= 0;
+            const int64_t ro = ok ? (int64_t)row * s.H + h : 0;
+            if (np < 3)
+                merge_rows<D, 3, 1>(a, &ro, &ok, np, sl);
+            else if (ok)
+                merge_row_any<D>(a.part_ml, a.part_o, a.O, a.lse, a.nseg, a.nsplit, ro, np, sl);
         }
     }
 }
 
 template <int D, int MT, int ST, int NW, int NS>
-cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyArgs& a, int gslots, bool pdl,
-                     cudaStream_t st) {
+cudaError_t launch_t(const TMaps& tm, const VerifyArgs& a, int gslots, bool pdl, cudaStream_t st) {
     using Lay = FusedLayout<D, MT, ST, NW, NS>;
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
     static bool configured = false;
@@ -1002,7 +1022,7 @@ cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyA
     }
     cfg.attrs = attr;
     cfg.numAttrs = n;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, verify_kernel<D, MT, ST, NW, NS>, tk, tv, a);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, verify_kernel<D, MT, ST, NW, NS>, tm, a);
     ripe_count_launch();
     return e;
 }
@@ -1011,27 +1031,28 @@ cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyA
 
 bool fused_supported(int dtype, int d) { return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128); }
 
-cudaError_t launch_fused(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt, bool pdl,
-                         cudaStream_t st) {
-    const CUtensorMap& tk = *reinterpret_cast<const CUtensorMap*>(tmK);
-    const CUtensorMap& tv = *reinterpret_cast<const CUtensorMap*>(tmV);
+cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int mt, bool pdl, cudaStream_t st) {
+    const TMaps& tm = *reinterpret_cast<const TMaps*>(tmaps);
     const int d = a.s.d;
     // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
     if (mt == 1) {
-        if (d == 64) return launch_t<64, 1, 4, 6, 3>(tk, tv, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 1, 3, 6, 2>(tk, tv, a, gslots, pdl, st);
-        if (d == 128) return launch_t<128, 1, 2, 5, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 64) return launch_t<64, 1, 4, 6, 3>(tm, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 1, 2, 8, 2>(tm, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 1, 2, 5, 2>(tm, a, gslots, pdl, st);
     } else {
-        if (d == 64) return launch_t<64, 2, 3, 6, 2>(tk, tv, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 2, 2, 4, 2>(tk, tv, a, gslots, pdl, st);
-        if (d == 128) return launch_t<128, 2, 2, 1, 2>(tk, tv, a, gslots, pdl, st);
+        if (d == 64) return launch_t<64, 2, 3, 6, 2>(tm, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 2, 2, 4, 2>(tm, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 2, 2, 1, 2>(tm, a, gslots, pdl, st);
     }
     return cudaErrorInvalidValue;
 }
 
-// Tensor maps of the deep planes: 2-D [rows = L*Bmax*H*Tmax][d] bf16, box 32 x 64
-// with the 64-byte swizzle the MMA descriptors above expect.
-int make_deep_tensor_maps(ripe_cache_s* c) {
+// Tensor maps: 2-D [rows][d] bf16 views, 32-column boxes with the 64-byte swizzle
+// the kernel's shared-memory layouts expect.  Deep planes (rows = L*Bmax*H*Tmax)
+// in 64-row boxes (deep region) and 16-row boxes (window tiles at depth R); ring
+// planes (rows = L*Bmax*H*(R-1)*Wcap) in 16-row boxes.  Rows past the end of a
+// view read as zeros.
+int make_tensor_maps(ripe_cache_s* c) {
     typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1044,18 +1065,32 @@ int make_deep_tensor_maps(ripe_cache_s* c) {
             return -1;
         encode = reinterpret_cast<EncodeFn>(fn);
     }
-    const cuuint64_t rows = (cuuint64_t)c->L * c->Bmax * c->H * c->Tmax;
-    if (rows >= (1ull << 31)) return -2;
-    const cuuint64_t dims[2] = {(cuuint64_t)c->d, rows};
+    static_assert(sizeof(TMaps) == sizeof(c->tmaps), "tensor map bundle");
+    const cuuint64_t deep_rows = (cuuint64_t)c->L * c->Bmax * c->H * c->Tmax;
+    const cuuint64_t ring_rows = (cuuint64_t)c->L * c->Bmax * c->H * (c->R - 1) * c->Wcap;
+    if (deep_rows >= (1ull << 31) || ring_rows >= (1ull << 31)) return -2;
     const cuuint64_t strides[1] = {(cuuint64_t)c->d * 2};
-    const cuuint32_t box[2] = {32, (cuuint32_t)kN};
     const cuuint32_t estr[2] = {1, 1};
-    CUtensorMap* maps[2] = {reinterpret_cast<CUtensorMap*>(c->tmap_k), reinterpret_cast<CUtensorMap*>(c->tmap_v)};
-    void* bases[2] = {c->kdeep, c->vdeep};
-    for (int i = 0; i < 2; ++i) {
-        CUresult r = encode(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, bases[i], dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    struct Spec {
+        void* base;
+        cuuint64_t rows;
+        cuuint32_t box_rows;
+    };
+    // With no ring planes (R = 1) the ring maps are never used; they alias the deep planes.
+    const bool ring = ring_rows > 0;
+    const Spec spec[6] = {{c->kdeep, deep_rows, (cuuint32_t)kN},
+                          {c->vdeep, deep_rows, (cuuint32_t)kN},
+                          {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
+                          {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
+                          {c->kdeep, deep_rows, (cuuint32_t)kWinKeys},
+                          {c->vdeep, deep_rows, (cuuint32_t)kWinKeys}};
+    for (int i = 0; i < 6; ++i) {
+        const cuuint64_t dims[2] = {(cuuint64_t)c->d, spec[i].rows};
+        const cuuint32_t box[2] = {32, spec[i].box_rows};
+        CUresult r = encode(reinterpret_cast<CUtensorMap*>(c->tmaps[i]), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                            spec[i].base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return -3;
     }
     return 0;

@@ -22,10 +22,10 @@ struct ripe_cache_s {
     // Verify scratch (per-split partial results), grown on demand.
     void* work;
     size_t work_bytes;
-    // TMA descriptors (CUtensorMap) of the deep K and V planes, when the tensor-core
-    // deep kernel serves this cache (bf16, d in {64, 96, 128}).
-    alignas(64) unsigned char tmap_k[128];
-    alignas(64) unsigned char tmap_v[128];
+    // TMA descriptors (CUtensorMap), when the fused sm_100a kernel serves this cache
+    // (bf16, d in {64, 96, 128}): deep K, V planes in 64-row boxes (deep region),
+    // ring K, V planes and deep K, V planes in 16-row boxes (window tiles).
+    alignas(64) unsigned char tmaps[6][128];
     bool tc_ready;
 };
 

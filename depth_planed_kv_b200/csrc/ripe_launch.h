@@ -34,9 +34,9 @@ void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit
 
 struct VerifyArgs;
 bool fused_supported(int dtype, int d);
-cudaError_t launch_fused(const void* tmK, const void* tmV, const VerifyArgs& a, int gslots, int mt, bool pdl,
-                         cudaStream_t st);
-int make_deep_tensor_maps(ripe_cache_s* c);
+cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int mt, bool pdl, cudaStream_t st);
+// The six tensor maps of the fused kernel (0 on success).
+int make_tensor_maps(ripe_cache_s* c);
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
                           const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,

@@ -453,7 +453,7 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     if (plan.fused) {
         // The whole call in one kernel; programmatic dependent launch lets its
         // prologue overlap the tail of the previous kernel in the stream.
-        e = launch_fused(c->tmap_k, c->tmap_v, a, plan.gslots, plan.mt, true, st);
+        e = launch_fused(c->tmaps, a, plan.gslots, plan.mt, true, st);
         if (e != cudaSuccess) return e;
     } else {
         const int keys_ub = plan.chunk > win_ub ? plan.chunk : win_ub;
