@@ -71,15 +71,13 @@ struct FusedLayout {
     static constexpr int NCH = D / 32;               // 64-byte column chunks of the head dim
     static constexpr int Q_BYTES = MT * NCH * 8192;  // 128 rows x 64 B per chunk
     static constexpr int KV_STAGE = NCH * 4096;      // 64 keys x 64 B per chunk
-    static constexpr int P_BUF = 2 * 8192;           // one M tile: 2 chunks of 32 keys
     static constexpr int WBOX = kWinKeys * 64;       // one 16-row x 64-byte window box
     static constexpr int WKV = NCH * WBOX;           // K (or V) of one window tile
     static constexpr int WSTAGE = 2 * WKV;           // K boxes, then V boxes
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
-    static constexpr int OFF_P = OFF_V + ST * KV_STAGE;
-    static constexpr int OFF_W = OFF_P + 2 * MT * P_BUF;
+    static constexpr int OFF_W = OFF_V + ST * KV_STAGE;
     static constexpr int OFF_BAR = OFF_W + NW * NS * WSTAGE;
     // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
     static constexpr int NBAR = 1 + 3 * ST + 7;
@@ -310,7 +308,6 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
     uint8_t* sQ = sm + Lay::OFF_Q;
     uint8_t* sK = sm + Lay::OFF_K;
     uint8_t* sV = sm + Lay::OFF_V;
-    uint8_t* sP = sm + Lay::OFF_P;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::OFF_BAR);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
@@ -464,9 +461,9 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
             } else if (warp == 5) {
                 // ------------------------------------------------ MMA issuer
                 if (lane == 0) {
-                    const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV), p0 = smem_u32(sP);
+                    const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV);
                     auto issue_pv = [&](int t) -> bool {
-                        const int st = t % ST, pb = t & 1, it_in_rt = t % ntiles;
+                        const int st = t % ST, pb = t & 1, it_in_rt = t % ntiles;  // P of tile t in S buffer pb
                         if (!mbar_wait(p_full + pb, (t >> 1) & 1, abort_flag, s.err)) return false;
                         if (!mbar_wait(v_full + st, (t / ST) & 1, abort_flag, s.err)) return false;
                         tc_fence_after();
@@ -474,12 +471,10 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                         for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
                             for (int ks = 0; ks < kN / 16; ++ks) {
-                                const uint64_t ad = smem_desc(p0 + (pb * MT + mt) * Lay::P_BUF + (ks >> 1) * 8192 +
-                                                                  (ks & 1) * 32, 16, 512, kLayoutSwizzle64B);
                                 const uint64_t bd = smem_desc(v0 + st * Lay::KV_STAGE + ks * 1024, kN * 64, 512,
                                                               kLayoutSwizzle64B);
-                                mma_bf16(tmem + Lay::O_COL(mt), ad, bd, IDESC_PV,
-                                         (it_in_rt > 0 || ks > 0) ? 1u : 0u);
+                                mma_bf16_ts(tmem + Lay::O_COL(mt), tmem + Lay::S_COL(mt, pb) + ks * 8, bd, IDESC_PV,
+                                            (it_in_rt > 0 || ks > 0) ? 1u : 0u);
                             }
                         }
                         mma_commit(kv_empty + st);
@@ -568,10 +563,6 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                     tc_fence_after();
                     const int key0 = G.key_begin + i * kN;
                     const int nvalid = min(kN, G.key_end - key0);
-                    if (it >= 2 && !warp_wait(pv_done + sb, ((it - 2) >> 1) & 1, abort_flag, s.err)) {
-                        ok = false;
-                        break;
-                    }
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
                         float sc[kN];
@@ -602,27 +593,21 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                             alpha = ex2(m[mt] - mn);
                             m[mt] = mn;
                         }
-                        // p = 2^(s*scale*log2e - m): one FMA and one ex2 per score.
+                        // p = 2^(s*scale*log2e - m): one FMA and one ex2 per score.  P (bf16
+                        // pairs) goes back into the first 32 columns of this tile's S buffer,
+                        // the A operand of P V (the next write of the buffer, QK of tile
+                        // it+2, follows P V of this tile in the MMA order).
                         const float nm = -m[mt];
                         float s4[4] = {0.f, 0.f, 0.f, 0.f};
-                        uint8_t* prow = sP + (sb * MT + mt) * Lay::P_BUF + t * 64;
+                        float pw[kN / 2];
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-                            for (int gq = 0; gq < 4; ++gq) {
-                                uint32_t w[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const float x0 = ex2(fmaf(sc[c * 32 + gq * 8 + 2 * e], c2, nm));
-                                    const float x1 = ex2(fmaf(sc[c * 32 + gq * 8 + 2 * e + 1], c2, nm));
-                                    s4[e] += x0 + x1;
-                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
-                                    w[e] = *reinterpret_cast<uint32_t*>(&b2);
-                                }
-                                *reinterpret_cast<uint4*>(prow + c * 8192 + ((gq ^ ((t >> 1) & 3)) << 4)) =
-                                    make_uint4(w[0], w[1], w[2], w[3]);
-                            }
+                        for (int c = 0; c < kN / 2; ++c) {
+                            const float x0 = ex2(fmaf(sc[2 * c], c2, nm));
+                            const float x1 = ex2(fmaf(sc[2 * c + 1], c2, nm));
+                            s4[c & 3] += x0 + x1;
+                            pw[c] = __uint_as_float(pack_bf16(x0, x1));
                         }
+                        tmem_st32(lane_addr + Lay::S_COL(mt, sb), pw);
                         l[mt] = l[mt] * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
                         if (i > 0 && __any_sync(0xffffffffu, grow)) {
                             // O holds this row tile's earlier tiles: rescale it once PV(it-1) is done
@@ -645,7 +630,7 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                         }
                     }
                     if (!ok) break;
-                    fence_proxy_async_smem();
+                    tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(p_full + sb);
                     if (i == ntiles - 1) {
@@ -655,11 +640,13 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                             break;
                         }
                         tc_fence_after();
-                        // The P buffers are free here (every PV of the row tile is done):
-                        // each warp passes its 32 rows through them 32 columns at a time
-                        // and stores 128-byte row pieces (coalesced).
+                        // Every MMA of the row tile is done, so this warp's own Q rows are
+                        // free (other warps may already stage their next Q rows): the warp
+                        // passes its rows through the first 2 KB of them, 8 rows x 32
+                        // columns at a time, and stores 128-byte row pieces (coalesced).
                         constexpr int OSTR = 32 * 4 + 16;
-                        uint8_t* ostage = sP + warp * 32 * OSTR;
+                        static_assert(8 * OSTR <= 2048, "epilogue staging");
+                        uint8_t* ostage = sQ + warp * 2048;
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             const int row = rows[mt];
@@ -670,20 +657,25 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                                 float o[32];
                                 tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
                                 tmem_wait_ld();
-                                float4* d4 = reinterpret_cast<float4*>(ostage + lane * OSTR);
 #pragma unroll
-                                for (int c = 0; c < 8; ++c)
-                                    d4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-                                __syncwarp();
+                                for (int part = 0; part < 4; ++part) {
+                                    if ((lane >> 3) == part) {
+                                        float4* d4 = reinterpret_cast<float4*>(ostage + (lane & 7) * OSTR);
 #pragma unroll
-                                for (int e0 = 0; e0 < 32 * 8; e0 += 32) {
-                                    const int e = e0 + lane, kr = e >> 3, c4 = e & 7;
-                                    const int64_t pk = __shfl_sync(0xffffffffu, pi, kr);
-                                    if (pk >= 0)
-                                        reinterpret_cast<float4*>(a.part_o + pk * D + c0)[c4] =
-                                            *reinterpret_cast<const float4*>(ostage + kr * OSTR + c4 * 16);
+                                        for (int c = 0; c < 8; ++c)
+                                            d4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                                    }
+                                    __syncwarp();
+#pragma unroll
+                                    for (int e0 = 0; e0 < 8 * 8; e0 += 32) {
+                                        const int e = e0 + lane, kr = e >> 3, c4 = e & 7;
+                                        const int64_t pk = __shfl_sync(0xffffffffu, pi, part * 8 + kr);
+                                        if (pk >= 0)
+                                            reinterpret_cast<float4*>(a.part_o + pk * D + c0)[c4] =
+                                                *reinterpret_cast<const float4*>(ostage + kr * OSTR + c4 * 16);
+                                    }
+                                    __syncwarp();
                                 }
-                                __syncwarp();
                             }
                         }
                         tc_fence_before();
@@ -1036,13 +1028,13 @@ cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int
     const int d = a.s.d;
     // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
     if (mt == 1) {
-        if (d == 64) return launch_t<64, 1, 4, 6, 3>(tm, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 1, 2, 8, 2>(tm, a, gslots, pdl, st);
-        if (d == 128) return launch_t<128, 1, 2, 5, 2>(tm, a, gslots, pdl, st);
+        if (d == 64) return launch_t<64, 1, 4, 8, 3>(tm, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 1, 3, 8, 2>(tm, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 1, 3, 5, 2>(tm, a, gslots, pdl, st);
     } else {
-        if (d == 64) return launch_t<64, 2, 3, 6, 2>(tm, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 2, 2, 4, 2>(tm, a, gslots, pdl, st);
-        if (d == 128) return launch_t<128, 2, 2, 1, 2>(tm, a, gslots, pdl, st);
+        if (d == 64) return launch_t<64, 2, 4, 8, 2>(tm, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 2, 3, 6, 2>(tm, a, gslots, pdl, st);
+        if (d == 128) return launch_t<128, 2, 2, 4, 2>(tm, a, gslots, pdl, st);
     }
     return cudaErrorInvalidValue;
 }
