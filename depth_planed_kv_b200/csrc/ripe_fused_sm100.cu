@@ -37,6 +37,8 @@
 // 16 keys in the same 64-byte-swizzled 32-column boxes (conflict-free ldmatrix).
 #include <cuda.h>
 
+#include <cstring>
+
 #include "ripe_launch.h"
 #include "ripe_verify.cuh"
 #include "sm100_ptx.cuh"
@@ -51,9 +53,10 @@ constexpr int kWinKeys = 16;  // keys per window tile (the M of an m16n8k16 tile
 constexpr int kRowTable = 512;  // group rows whose Q/O row index is tabulated in shared memory
 
 // Tensor maps of one launch: deep K, V in 64-row boxes; ring K, V and deep K, V
-// in 16-row boxes (all 32 columns wide, 64-byte swizzle).
+// in 16-row boxes; Q of this call as [rows][H][d] in 128-row boxes of one head (all
+// 32 columns wide, 64-byte swizzle).  The first six belong to the cache.
 struct TMaps {
-    CUtensorMap dk, dv, wk, wv, rk, rv;
+    CUtensorMap dk, dv, wk, wv, rk, rv, q;
 };
 
 // One branch of the group: its rows, its offset among the group's rows, its
@@ -79,8 +82,9 @@ struct FusedLayout {
     static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
     static constexpr int OFF_W = OFF_V + ST * KV_STAGE;
     static constexpr int OFF_BAR = OFF_W + NW * NS * WSTAGE;
-    // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain
-    static constexpr int NBAR = 1 + 3 * ST + 7;
+    // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain,
+    // epi_done
+    static constexpr int NBAR = 1 + 3 * ST + 8;
     static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;  // one per window stage
     static constexpr int OFF_MISC = OFF_WBAR + NW * NS * 8;
     static constexpr int OFF_BT = OFF_MISC + 64;
@@ -317,6 +321,7 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
     uint64_t* p_full = s_full + 2;
     uint64_t* pv_done = s_full + 4;
     uint64_t* drain = s_full + 6;
+    uint64_t* epi_done = s_full + 7;  // the softmax warps' epilogue staging is finished
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 4);
     GroupInfo* gi = reinterpret_cast<GroupInfo*>(sm + Lay::OFF_MISC + 16);
@@ -340,6 +345,7 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
             mbar_init(pv_done + i, 1);
         }
         mbar_init(drain, 1);
+        mbar_init(epi_done, 4);
         for (int i = 0; i < NW * NS; ++i) mbar_init(reinterpret_cast<uint64_t*>(sm + Lay::OFF_WBAR) + i, 32);
         *abort_flag = 0;
         fence_barrier_init();
@@ -427,6 +433,9 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
     const int ntiles = G.key_end > G.key_begin ? (G.key_end - G.key_begin + kN - 1) / kN : 0;
     const int nrt = (G.nrows + RT - 1) / RT;
     const int total_it = ntiles * nrt;
+    // All-depths groups (k tokens x R depths of one sequence) are one block of Q rows.
+    const int q_block =
+        (a.q_tma && !a.ba.table && G.nrows == a.ba.k * s.R) ? g * a.ba.k * s.R : -1;
 
     if (warp < 6) {
         if (total_it > 0) {
@@ -528,7 +537,32 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                 bool ok = true;
                 for (int it = 0; it < total_it && ok; ++it) {
                     const int i = it % ntiles, rt = it / ntiles, sb = it & 1;
-                    if (i == 0) {
+                    if (i == 0 && q_block >= 0) {
+                        // The group's rows are one block of Q (all-depths form): M row t is
+                        // Q row q_block + t; one thread loads the row tile by TMA, once the
+                        // previous row tile's epilogue has left the Q buffer.
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const int rl = rt * RT + mt * 128 + t;
+                            rows[mt] = rl < G.nrows ? q_block + rl : -1;
+                            m[mt] = -INFINITY;
+                            l[mt] = 0.f;
+                        }
+                        if (t == 0) {
+                            bool go = rt == 0 || mbar_wait(epi_done, (rt - 1) & 1, abort_flag, s.err);
+                            if (go) {
+                                mbar_expect_tx(q_full, MT * NCH * 8192);
+#pragma unroll
+                                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                    for (int c = 0; c < NCH; ++c)
+                                        tma_load_3d(sQ + mt * NCH * 8192 + c * 8192, &tm.q, 32 * c, h,
+                                                    q_block + rt * RT + mt * 128, q_full);
+                            }
+                        } else {
+                            mbar_arrive(q_full);
+                        }
+                    } else if (i == 0) {
                         // Rows of this row tile (each thread finds its own); the warp copies
                         // its 32 rows' Q, 16 bytes per lane in row order (coalesced), into
                         // the swizzled K-major layout.
@@ -678,6 +712,10 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                                 }
                             }
                         }
+                        // The staging stores come before any later TMA write of the Q buffer.
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(epi_done);
                         tc_fence_before();
                     }
                 }
@@ -1021,10 +1059,43 @@ cudaError_t launch_t(const TMaps& tm, const VerifyArgs& a, int gslots, bool pdl,
 
 }  // namespace
 
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver (looked up once), or NULL.
+static EncodeFn encode_fn() {
+    static EncodeFn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && fn)
+            encode = reinterpret_cast<EncodeFn>(fn);
+    }
+    return encode;
+}
+
 bool fused_supported(int dtype, int d) { return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128); }
 
-cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int mt, bool pdl, cudaStream_t st) {
-    const TMaps& tm = *reinterpret_cast<const TMaps*>(tmaps);
+cudaError_t launch_fused(const void* tmaps, const VerifyArgs& args, int gslots, int mt, bool pdl, cudaStream_t st) {
+    // The cache's maps plus one of this call's Q, viewed as [rows][H][d]: boxes of
+    // 128 rows x 32 columns of one head (the stacked-query tile of the deep region).
+    TMaps tm;
+    memcpy(&tm, tmaps, 6 * sizeof(CUtensorMap));
+    VerifyArgs a = args;
+    a.q_tma = 0;
+    if (const EncodeFn encode = encode_fn()) {
+        const int d = a.s.d;
+        const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)a.s.H, (cuuint64_t)a.ba.nrows};
+        const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)a.s.H * d * 2};
+        const cuuint32_t box[3] = {32, 1, 128};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<char*>(a.Q), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            a.q_tma = 1;
+    }
     const int d = a.s.d;
     // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
     if (mt == 1) {
@@ -1045,19 +1116,9 @@ cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int
 // planes (rows = L*Bmax*H*(R-1)*Wcap) in 16-row boxes.  Rows past the end of a
 // view read as zeros.
 int make_tensor_maps(ripe_cache_s* c) {
-    typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static EncodeFn encode = nullptr;
-    if (!encode) {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || !fn)
-            return -1;
-        encode = reinterpret_cast<EncodeFn>(fn);
-    }
-    static_assert(sizeof(TMaps) == sizeof(c->tmaps), "tensor map bundle");
+    const EncodeFn encode = encode_fn();
+    if (!encode) return -1;
+    static_assert(sizeof(TMaps) == sizeof(c->tmaps) + sizeof(CUtensorMap), "tensor map bundle");
     const cuuint64_t deep_rows = (cuuint64_t)c->L * c->Bmax * c->H * c->Tmax;
     const cuuint64_t ring_rows = (cuuint64_t)c->L * c->Bmax * c->H * (c->R - 1) * c->Wcap;
     if (deep_rows >= (1ull << 31) || ring_rows >= (1ull << 31)) return -2;

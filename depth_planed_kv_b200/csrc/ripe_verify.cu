@@ -445,6 +445,7 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     a.scale_log2 = scale * 1.4426950408889634f;
     a.nsplit = plan.nsplit; a.chunk = plan.chunk; a.nseg = plan.nsplit + 1;
     a.nrowchunks = plan.nrowchunks;
+    a.q_tma = 0;
     char* wb = reinterpret_cast<char*>(work);
     a.part_ml = reinterpret_cast<float2*>(wb);
     a.part_o = reinterpret_cast<float*>(wb + verify_ml_bytes(ba.nrows, c->H, a.nseg));

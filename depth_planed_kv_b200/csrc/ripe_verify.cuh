@@ -16,6 +16,7 @@ struct VerifyArgs {
     int nrowchunks;           // row chunks per branch in the CUDA-core kernel
     float2* part_ml;          // [nrows][H][nseg] (m in log2 units, l)
     float* part_o;            // [nrows][H][nseg][d]
+    int q_tma;                // fused kernel: a tensor map of Q came with the launch
 };
 
 // Deep splits that hold keys for a sequence whose deep region has A keys.
