@@ -196,6 +196,32 @@ def cpu_baseline(wl, budget_s=10.0):
             "query_rows_per_s": done_rows / spent}
 
 
+# ---------------------------------------------------------------- multi-rank host logic
+# One process per GPU; ranks verify disjoint sequences (their own synthetic stores)
+# and exchange nothing on the data path: NCCL (gloo on CPU) serves only the barrier
+# and the max-over-ranks step time.
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Seed of the synthetic store of `rank` (each rank holds different sequences)."""
+    return seed + 17 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: every rank calls this, in the same order."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(bytes_per_step_per_rank: float, world: int, steps: int, ms_max: float) -> float:
+    """GB/s of all ranks together over the slowest rank's time (weak scaling)."""
+    return bytes_per_step_per_rank * world * steps / (ms_max / 1e3) / 1e9
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -273,7 +299,8 @@ def main():
     wl = S.huginn()
     nrep = 2
     cache = RipeCache(wl.layers, wl.R, wl.H, wl.d, wl.W, wl.Tmax, nrep, wl.kmax, torch.bfloat16)
-    cache.ripe_synth_fill(list(range(nrep)), [wl.ctx] * nrep, wl.seed + 17 * rank, S.coef_table(wl.decay, wl.R))
+    cache.ripe_synth_fill(list(range(nrep)), [wl.ctx] * nrep, shard_seed(wl.seed, rank),
+                          S.coef_table(wl.decay, wl.R))
     ids = [torch.tensor([s], dtype=torch.int32, device="cuda") for s in range(nrep)]
     for s in range(nrep):
         cache.ripe_evict(ids[s])
@@ -325,12 +352,6 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for i in range(warmup):
         step(i)
@@ -358,7 +379,7 @@ def main():
         torch.cuda.synchronize()
         n1 = launch_count()
     ms = e0.elapsed_time(e1)
-    ms_max = max_over_ranks(ms)
+    ms_max = max_over_ranks(ms, world, "cuda")
     # Kernel duration for the roofline: a separate pass with an event pair around every
     # call (events between calls stop consecutive calls from overlapping, so this pass
     # is not the step time).
@@ -381,10 +402,10 @@ def main():
         step_e2e(i)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, "cuda")
 
-    value = bytes_step * world * args.steps / (ms_max / 1e3) / 1e9
-    e2e_value = bytes_step * world * args.steps / (e2e_ms / 1e3) / 1e9
+    value = whole_job_rate(bytes_step, world, args.steps, ms_max)
+    e2e_value = whole_job_rate(bytes_step, world, args.steps, e2e_ms)
     peak, peak_kind = measured_peak()
     # Average launch duration over the timed region: consecutive calls overlap their
     # prologues (programmatic dependent launch), so the region divided by its launches
