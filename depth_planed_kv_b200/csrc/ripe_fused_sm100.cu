@@ -72,7 +72,10 @@ struct GroupInfo {
 template <int D, int MT, int ST, int NW, int NS>
 struct FusedLayout {
     static constexpr int NCH = D / 32;               // 64-byte column chunks of the head dim
-    static constexpr int Q_BYTES = MT * NCH * 8192;  // 128 rows x 64 B per chunk
+    // With one M tile, Q lives in tensor memory (A operand of QK^T from TMEM); with two,
+    // TMEM is full and Q stays in shared memory (128 rows x 64 B per chunk).
+    static constexpr bool QT = MT == 1;
+    static constexpr int Q_BYTES = QT ? 0 : MT * NCH * 8192;
     static constexpr int KV_STAGE = NCH * 4096;      // 64 keys x 64 B per chunk
     static constexpr int WBOX = kWinKeys * 64;       // one 16-row x 64-byte window box
     static constexpr int WKV = NCH * WBOX;           // K (or V) of one window tile
@@ -81,7 +84,9 @@ struct FusedLayout {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
     static constexpr int OFF_W = OFF_V + ST * KV_STAGE;
-    static constexpr int OFF_BAR = OFF_W + NW * NS * WSTAGE;
+    static constexpr int OFF_OST = OFF_W + NW * NS * WSTAGE;  // epilogue staging (Q in TMEM)
+    static constexpr int OST_BYTES = QT ? 4 * 8 * (32 * 4 + 16) : 0;
+    static constexpr int OFF_BAR = OFF_OST + OST_BYTES;
     // barriers: q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain,
     // epi_done
     static constexpr int NBAR = 1 + 3 * ST + 8;
@@ -92,9 +97,10 @@ struct FusedLayout {
     static constexpr int BYTES = OFF_RT + kRowTable * 4;
     static constexpr int SMEM = BYTES + 1024;  // alignment slack
     static constexpr int THREADS = kDeepThreads + 32 * NW;
-    static constexpr uint32_t TMEM_COLS = MT == 1 ? 256 : 512;
+    static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
     static constexpr uint32_t O_COL(int mt) { return (uint32_t)(MT * 2 * kN + mt * 128); }
+    static constexpr uint32_t Q_COL = 2 * kN + 128;  // Q in TMEM (QT): D/2 columns
 };
 
 // Warp-uniform bounded wait: every lane waits, and all lanes agree on the outcome
@@ -511,11 +517,16 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
                                 const uint32_t off = (ks & 1) * 32;
-                                const uint64_t ad = smem_desc(q0 + mt * NCH * 8192 + (ks >> 1) * 8192 + off, 16,
-                                                              512, kLayoutSwizzle64B);
                                 const uint64_t bd = smem_desc(k0 + st * Lay::KV_STAGE + (ks >> 1) * 4096 + off, 16,
                                                               512, kLayoutSwizzle64B);
-                                mma_bf16(tmem + Lay::S_COL(mt, sb), ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+                                if constexpr (Lay::QT) {
+                                    mma_bf16_ts(tmem + Lay::S_COL(mt, sb), tmem + Lay::Q_COL + ks * 8, bd, IDESC_QK,
+                                                ks > 0 ? 1u : 0u);
+                                } else {
+                                    const uint64_t ad = smem_desc(q0 + mt * NCH * 8192 + (ks >> 1) * 8192 + off, 16,
+                                                                  512, kLayoutSwizzle64B);
+                                    mma_bf16(tmem + Lay::S_COL(mt, sb), ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+                                }
                             }
                         }
                         mma_commit(s_full + sb);
@@ -537,7 +548,34 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                 bool ok = true;
                 for (int it = 0; it < total_it && ok; ++it) {
                     const int i = it % ntiles, rt = it / ntiles, sb = it & 1;
-                    if (i == 0 && q_block >= 0) {
+                    if (i == 0 && Lay::QT) {
+                        // Q into tensor memory: each thread its own row (TMEM lane t), loaded
+                        // as 16-byte vectors and stored as D/2 columns of bf16 pairs.  The
+                        // previous row tile's QK^T are done (its epilogue waited for them).
+                        const int rl = rt * RT + t;
+                        const int row = q_block >= 0 ? (rl < G.nrows ? q_block + rl : -1)
+                                                     : group_row(rowtab, bt, G.nb, G.nrows, rl);
+                        rows[0] = row;
+                        m[0] = -INFINITY;
+                        l[0] = 0.f;
+                        const uint4* src = reinterpret_cast<const uint4*>(a.Q + ((int64_t)(row >= 0 ? row : 0) * s.H + h) * D * 2);
+#pragma unroll
+                        for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                const uint4 x = row >= 0 ? __ldg(src + c0 / 4 + v) : make_uint4(0, 0, 0, 0);
+                                w[4 * v] = x.x;
+                                w[4 * v + 1] = x.y;
+                                w[4 * v + 2] = x.z;
+                                w[4 * v + 3] = x.w;
+                            }
+                            tmem_st16(lane_addr + Lay::Q_COL + c0, w);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(q_full);
+                    } else if (i == 0 && q_block >= 0) {
                         // The group's rows are one block of Q (all-depths form): M row t is
                         // Q row q_block + t; one thread loads the row tile by TMA, once the
                         // previous row tile's epilogue has left the Q buffer.
@@ -680,7 +718,7 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                         // columns at a time, and stores 128-byte row pieces (coalesced).
                         constexpr int OSTR = 32 * 4 + 16;
                         static_assert(8 * OSTR <= 2048, "epilogue staging");
-                        uint8_t* ostage = sQ + warp * 2048;
+                        uint8_t* ostage = Lay::QT ? sm + Lay::OFF_OST + warp * 8 * OSTR : sQ + warp * 2048;
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             const int row = rows[mt];
@@ -1100,7 +1138,7 @@ cudaError_t launch_fused(const void* tmaps, const VerifyArgs& args, int gslots, 
     // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
     if (mt == 1) {
         if (d == 64) return launch_t<64, 1, 4, 8, 3>(tm, a, gslots, pdl, st);
-        if (d == 96) return launch_t<96, 1, 3, 8, 2>(tm, a, gslots, pdl, st);
+        if (d == 96) return launch_t<96, 1, 3, 8, 3>(tm, a, gslots, pdl, st);
         if (d == 128) return launch_t<128, 1, 3, 5, 2>(tm, a, gslots, pdl, st);
     } else {
         if (d == 64) return launch_t<64, 2, 4, 8, 2>(tm, a, gslots, pdl, st);
