@@ -35,6 +35,20 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+}  // namespace
+
+bool stream_capturing(cudaStream_t st) {
+    if (!st) return false;  // the legacy default stream is never captured
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return cs != cudaStreamCaptureStatusNone;
+}
+
+namespace {
+
 struct Layout {
     size_t kdeep, vdeep, kwin, vwin, len, ws, err, total;
 };
@@ -120,7 +134,9 @@ int verify_common(ripe_cache_s* c, int layer, const BranchArgs& ba, const void* 
     if (lse && ((uintptr_t)lse & 3u)) return fail(RIPE_ERR_UNALIGNED, "lse must be 4-byte aligned");
     if (!(scale == scale) || isinf(scale)) return fail(RIPE_ERR_INVALID_ARG, "scale is not finite");
     if (scale == 0.f) scale = 1.0f / sqrtf((float)c->d);
-    const VerifyPlan plan = plan_verify(c, ba.nbranch, ba.nrows, ba.max_ntok, ba.table == nullptr);
+    // A captured launch replays while the sequences grow: its plan covers Tmax.
+    const VerifyPlan plan = plan_verify(c, ba.nbranch, ba.nrows, ba.max_ntok, ba.table == nullptr,
+                                        stream_capturing(st));
     int rc = ensure_workspace(c, plan.work_bytes, st);
     if (rc != RIPE_OK) return rc;
     cudaError_t e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, c->work, st);
@@ -246,10 +262,12 @@ int ripe_append(ripe_cache_t c, const int32_t* seq_ids, const int32_t* n_acc, in
     if (nseq == 0) return RIPE_OK;
     if (!seq_ids || !n_acc || !K || !V) return fail(RIPE_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned16(K) || !aligned16(V)) return fail(RIPE_ERR_UNALIGNED, "K and V must be 16-byte aligned");
-    cudaError_t e = launch_append(c, seq_ids, n_acc, nseq, K, V, kmax_in, as_stream(stream));
+    const cudaStream_t st = as_stream(stream);
+    cudaError_t e = launch_append(c, seq_ids, n_acc, nseq, K, V, kmax_in, st);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    // The host's bound on the lengths; a captured append may replay any number of times.
     const int64_t ub = (int64_t)c->len_ub + kmax_in;
-    c->len_ub = (int)(ub < c->Tmax ? ub : c->Tmax);
+    c->len_ub = stream_capturing(st) ? c->Tmax : (int)(ub < c->Tmax ? ub : c->Tmax);
     return RIPE_OK;
 }
 
@@ -313,8 +331,10 @@ int ripe_reserve_workspace(ripe_cache_t c, int max_rows) {
     int rc = check_cache(c);
     if (rc != RIPE_OK) return rc;
     if (max_rows < 0) return fail(RIPE_ERR_INVALID_ARG, "max_rows < 0");
-    const int nbranch = max_rows;  // upper bound: at least one row per branch
-    const VerifyPlan plan = plan_verify(c, nbranch, max_rows, c->kmax, false);
+    // The most scratch a call of up to max_rows rows can take under capture: the
+    // fewest branches and tokens per branch give the most splits, and captured
+    // calls plan for Tmax.
+    const VerifyPlan plan = plan_verify(c, 1, max_rows, 1, false, true);
     return ensure_workspace(c, plan.work_bytes, nullptr);
 }
 

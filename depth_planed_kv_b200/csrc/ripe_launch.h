@@ -25,10 +25,18 @@ struct VerifyPlan {
     bool fused;        // the whole call in the sm_100a fused kernel (tcgen05 deep region)
     int mt;            // M tiles (of 128 rows) per fused CTA
     int gslots;        // fused CTAs along the sequence-group axis
+    int a_ub;          // bound on the deep region's length the splits cover
+    int win_ub;        // bound on a branch's window + block keys (CUDA-core kernel)
     size_t work_bytes; // scratch needed
 };
 
-VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths);
+// `capacity`: plan for every length the store can hold (Tmax), not for the host's
+// bound on the current lengths -- for launches captured into a CUDA graph, which
+// replay while the sequences grow.
+VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
+                       bool capacity);
+// True while `st` is being captured into a CUDA graph.
+bool stream_capturing(cudaStream_t st);
 // Re-plan with `nsplit` deep splits (chunk and scratch size follow).
 void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit);
 

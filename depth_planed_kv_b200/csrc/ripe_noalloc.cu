@@ -72,7 +72,8 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
     ba.nbranch = nbranch;
     ba.nrows = nrows;
     ba.max_ntok = c->kmax;
-    VerifyPlan plan = plan_verify(c, nbranch, nrows, c->kmax, false);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    VerifyPlan plan = plan_verify(c, nbranch, nrows, c->kmax, false, stream_capturing(st));
     // Fewer, longer deep splits until the partial results fit the fixed array.
     while (plan.work_bytes > kStaticScratchBytes && plan.nsplit > 1) plan_set_splits(plan, c, nrows, plan.nsplit / 2);
     if (scratch_needed) *scratch_needed = plan.work_bytes;
@@ -83,8 +84,7 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
     cudaError_t e = static_scratch_address(&work);
     if (e != cudaSuccess)
         return ripe_fail(RIPE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-    e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, work,
-                      reinterpret_cast<cudaStream_t>(stream));
+    e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, work, st);
     if (e != cudaSuccess) return ripe_fail(RIPE_ERR_CUDA, "verify launch: %s", cudaGetErrorString(e));
     return RIPE_OK;
 }

@@ -392,12 +392,16 @@ cudaError_t launch_seg(const VerifyArgs& a, int seg_first, int seg_count, int nb
 
 }  // namespace
 
-VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths) {
+VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
+                       bool capacity) {
     VerifyPlan p{};
     p.max_ntok = max_ntok;
     p.nrowchunks = (max_ntok + kRowsPerCta - 1) / kRowsPerCta;
     if (p.nrowchunks < 1) p.nrowchunks = 1;
-    const int A_ub = c->len_ub < c->Tmax ? c->len_ub : c->Tmax;
+    const int len_ub = capacity ? c->Tmax : c->len_ub;
+    const int A_ub = len_ub < c->Tmax ? len_ub : c->Tmax;
+    p.a_ub = A_ub;
+    p.win_ub = (len_ub < c->Wcap ? len_ub : c->Wcap) + max_ntok;
     p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
     int64_t ns;
     if (p.fused) {
@@ -424,7 +428,7 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
 }
 
 void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit) {
-    const int A_ub = c->len_ub < c->Tmax ? c->len_ub : c->Tmax;
+    const int A_ub = p.a_ub;
     const int align = p.fused ? 64 : 32;  // deep tile of the fused kernel / key tile of the CUDA-core kernel
     p.nsplit = nsplit;
     int chunk = (A_ub + nsplit - 1) / nsplit;
@@ -450,7 +454,7 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     a.part_ml = reinterpret_cast<float2*>(wb);
     a.part_o = reinterpret_cast<float*>(wb + verify_ml_bytes(ba.nrows, c->H, a.nseg));
     cudaError_t e;
-    const int win_ub = (c->len_ub < c->Wcap ? c->len_ub : c->Wcap) + plan.max_ntok;
+    const int win_ub = plan.win_ub;
     if (plan.fused) {
         // The whole call in one kernel; programmatic dependent launch lets its
         // prologue overlap the tail of the previous kernel in the stream.

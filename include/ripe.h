@@ -135,6 +135,9 @@ int ripe_cache_reset(ripe_cache_t cache, const int32_t* seq_ids_dev, int nseq,
  *   kmax_in >= 1 (a prefill may exceed the cache's kmax: only the last Wcap
  *   positions then keep planes 1..R-1).  Sequence ids in one call must be distinct.
  * A sequence whose append would pass Tmax is skipped (RIPE_DEVERR_CAPACITY).
+ * The library keeps a host-side bound on the lengths (it plans verify launches
+ * from it); an append enqueued while the stream is captured into a CUDA graph
+ * may replay any number of times, so it raises that bound to Tmax.
  */
 int ripe_append(ripe_cache_t cache, const int32_t* seq_ids_dev, const int32_t* n_acc_dev, int nseq,
                 const void* K, const void* V, int kmax_in, ripe_stream_t stream);
@@ -177,6 +180,9 @@ int ripe_truncate(ripe_cache_t cache, const int32_t* seq_ids_dev, const int32_t*
  * a call that needs more than it holds grows it (a cudaMalloc), which returns
  * RIPE_ERR_CAPTURING if the stream is being captured -- call
  * ripe_reserve_workspace first in that case.
+ * CUDA graphs: a call enqueued while the stream is being captured is planned
+ * for every length the cache can hold (its deep-region splits cover Tmax), so
+ * the captured launch stays exact when replayed after the sequences have grown.
  */
 int ripe_verify_attn(ripe_cache_t cache, int layer, const ripe_branch_t* branches_dev, int nbranch,
                      int nrows, const void* Q, const void* Kblk, const void* Vblk,
@@ -225,7 +231,8 @@ int ripe_verify_attn_noalloc(ripe_cache_t cache, int layer, const ripe_branch_t*
                              const int32_t* ctx_len_dev, float scale, void* O, float* lse,
                              ripe_stream_t stream, size_t* scratch_needed);
 
-/* Pre-size the verify scratch for calls with up to max_rows rows (before stream capture). */
+/* Pre-size the verify scratch for any call of up to max_rows rows enqueued under
+ * stream capture (the largest split count such a call can get), before capture. */
 int ripe_reserve_workspace(ripe_cache_t cache, int max_rows);
 
 /*
