@@ -52,7 +52,7 @@ typedef enum {
     RIPE_ERR_OOM = 4,         /* device allocation failed */
     RIPE_ERR_CUDA = 5,        /* a CUDA runtime call failed */
     RIPE_ERR_DEVICE = 6,      /* the device error word was set (see ripe_get_device_error) */
-    RIPE_ERR_UNSUPPORTED = 7, /* shape or dtype this build has no kernel for */
+    RIPE_ERR_UNSUPPORTED = 7, /* shape or dtype the library has no kernel for */
     RIPE_ERR_CAPTURING = 8    /* the call would allocate while the stream is being captured */
 } ripe_status;
 

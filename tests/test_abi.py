@@ -55,7 +55,7 @@ def test_cache_bytes_matches_layout_and_memory_model():
     ((1, 0, 2, 16, 8, 64, 1, 4), 1),     # R
     ((1, 65, 2, 16, 8, 64, 1, 4), 1),
     ((1, 4, 2, 12, 8, 64, 1, 4), 3),     # d*2 not a multiple of 16 (bf16)
-    ((1, 4, 2, 256, 8, 64, 1, 4), 7),    # d above this build's kernels
+    ((1, 4, 2, 256, 8, 64, 1, 4), 7),    # d above the library's kernels
     ((1, 4, 2, 16, -1, 64, 1, 4), 1),    # W
     ((1, 4, 2, 16, 8, 64, 0, 4), 1),     # max_seqs
     ((1, 4, 2, 16, 8, 64, 1, 0), 1),     # kmax
