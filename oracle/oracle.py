@@ -150,6 +150,7 @@ class OracleStore:
       kwin/vwin   [L][Bmax][H][R-1][Wcap][d]    planes 1..R-1; position p in slot
                                                 p mod Wcap, Wcap = W + kmax
       length[b], wstart[b]                      committed length T_b, window start
+      rfloor[b]                                 ring floor (below)
     Positions ws_b <= p < T_b are live in the ring.
 
     append(seq b, n): positions T_b..T_b+n-1 get plane R in kdeep; of those, the
@@ -158,8 +159,25 @@ class OracleStore:
     T_b + n exceeds Tmax, or with n outside [0, kmax_in], are skipped and flagged.
     evict(seq b): ws_b = max(ws_b, T_b - W): positions leaving the window keep only
     their deepest plane, which kdeep already holds.
-    truncate(seq b, T'): rollback to a confirmed prefix (LoopSpec article, section
-    on the second branch): T_b = min(T_b, T'), ws_b = min(ws_b, T_b).
+
+    Ring floor rf_b: the lowest position whose ring slots still hold its own
+    planes 1..R-1 (positions below it were overwritten by later positions, or
+    never written by a long prefill).  append raises it to T_b - Wcap like ws_b,
+    but evict leaves it alone, so rf_b <= ws_b always.
+
+    truncate(seq b, T'): rollback to the confirmed prefix (LoopSpec article,
+    section on the second branch: a rejected early draft discards the dependent
+    work and decoding resumes from the confirmed prefix).  The target state is
+    the one a store that only ever saw the confirmed tokens reaches after its
+    evict at the confirmed length, as far as the ring still holds the planes:
+      T_b  = min(T_b, T')
+      rf_b = min(rf_b, T_b)
+      ws_b = min(ws_b, max(T_b - W, rf_b))
+    Positions that were evicted only because the rejected tokens pushed the
+    window forward come back into the window; positions whose ring slots the
+    rejected tokens overwrote cannot (with Wcap = W + kmax that happens only when
+    more than kmax positions are rolled back).  A truncate to T' >= T_b changes
+    nothing.
     """
 
     def __init__(self, L, R, H, d, W, Tmax, Bmax, kmax, np_dtype):
@@ -172,12 +190,14 @@ class OracleStore:
         self.vwin = np.zeros_like(self.kwin)
         self.length = np.zeros(Bmax, dtype=np.int32)
         self.wstart = np.zeros(Bmax, dtype=np.int32)
+        self.rfloor = np.zeros(Bmax, dtype=np.int32)
         self.flagged = False
 
     def reset(self, seq_ids):
         for b in seq_ids:
             self.length[b] = 0
             self.wstart[b] = 0
+            self.rfloor[b] = 0
 
     def append(self, seq_ids, n_acc, K, V):
         """K, V: [L][nseq][kmax_in][R][H][d]; plane index r-1 along axis 3."""
@@ -199,6 +219,7 @@ class OracleStore:
                     self.vwin[:, b, :, :, slot, :] = np.swapaxes(V[:, i, t, : self.R - 1], 1, 2)
             self.length[b] = T + n
             self.wstart[b] = max(int(self.wstart[b]), T + n - self.Wcap)
+            self.rfloor[b] = max(int(self.rfloor[b]), T + n - self.Wcap)
 
     def evict(self, seq_ids):
         for b in seq_ids:
@@ -206,9 +227,14 @@ class OracleStore:
 
     def truncate(self, seq_ids, new_len):
         for i, b in enumerate(seq_ids):
+            if int(new_len[i]) < 0:
+                self.flagged = True
+                continue
             T = min(int(self.length[b]), int(new_len[i]))
+            rf = min(int(self.rfloor[b]), T)
             self.length[b] = T
-            self.wstart[b] = min(int(self.wstart[b]), T)
+            self.rfloor[b] = rf
+            self.wstart[b] = min(int(self.wstart[b]), max(T - self.W, rf))
 
     def plane_view(self, layer: int, b: int):
         """What a verify reads for sequence b: the oracle's logical input dict."""

@@ -307,3 +307,106 @@ def test_generator_decay(key):
     dist = np.sqrt(((P - P[:, R - 1:R]) ** 2).sum(axis=(0, 2, 3)))
     ratios = dist[0:R - 2] / dist[1:R - 1]   # distance to plane R shrinks by `decay` per loop
     assert np.all(np.abs(ratios - decay) < 0.02)
+
+
+# --- rollback to the confirmed prefix (LoopSpec article, section on the second branch) -----
+
+def _block(rng, L, n, R, H, d):
+    return rng.standard_normal((L, 1, n, R, H, d)), rng.standard_normal((L, 1, n, R, H, d))
+
+
+def _all_depth_verify(st, seq, rng, R, H, d, k=3):
+    """Verify k fresh draft tokens at every depth over sequence seq of store st."""
+    nrows = k * R
+    Q = rng.standard_normal((nrows, H, d))
+    Kb = rng.standard_normal((nrows, H, d))
+    Vb = rng.standard_normal((nrows, H, d))
+    table = np.array([(seq, r, k, r - 1, R) for r in range(1, R + 1)], np.int32)
+    views = [st.plane_view(0, b) for b in range(st.Bmax)]
+    return OR.verify(views, table, Q, Kb, Vb, 1 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("W,kmax", [(8, 4), (4, 4), (2, 4), (0, 3), (1, 6), (16, 8)])
+def test_rollback_returns_to_confirmed_prefix(W, kmax):
+    """Decode steps that append a speculative block (all planes), evict, then roll
+    back to the accepted length leave a store that verifies exactly like one that
+    only ever appended the accepted tokens (append + evict per step).  Covers
+    windows longer and shorter than the speculative block (W >= n and W < n)."""
+    L, R, H, d, Tmax, B, seq = 1, 4, 2, 8, 200, 3, 1
+    rng = np.random.default_rng(1000 + 10 * W + kmax)
+    spec = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np.float64)
+    conf = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np.float64)
+    K0, V0 = _block(rng, L, 23, R, H, d)
+    for st in (spec, conf):
+        st.append([seq], [23], K0, V0)   # prefill: more than Wcap positions
+        st.evict([seq])
+    for step in range(12):
+        n = int(rng.integers(1, kmax + 1))
+        acc = int(rng.integers(0, n + 1))
+        K, V = _block(rng, L, n, R, H, d)
+        spec.append([seq], [n], K, V)
+        spec.evict([seq])
+        T_conf = int(conf.length[seq]) + acc
+        spec.truncate([seq], [T_conf])
+        conf.append([seq], [acc], K, V)  # the accepted tokens are the first acc of the block
+        conf.evict([seq])
+        assert int(spec.length[seq]) == int(conf.length[seq]) == T_conf
+        assert int(spec.wstart[seq]) == int(conf.wstart[seq]), (step, spec.wstart[seq], conf.wstart[seq])
+        vs, vc = spec.plane_view(0, seq), conf.plane_view(0, seq)
+        for key in ("Kd", "Vd", "Kw", "Vw"):
+            assert np.array_equal(vs[key], vc[key]), (step, key)
+        s = int(rng.integers(0, 2 ** 31))
+        Os, ls = _all_depth_verify(spec, seq, np.random.default_rng(s), R, H, d)
+        Oc, lc = _all_depth_verify(conf, seq, np.random.default_rng(s), R, H, d)
+        assert np.abs(Os - Oc).max() <= 1e-13 and np.abs(ls - lc).max() <= 1e-13
+
+
+def test_rollback_deeper_than_ring_keeps_only_intact_positions():
+    """Rolling back more than kmax positions: the rejected tokens overwrote ring
+    slots of confirmed positions, which then read at the deepest plane only.  Every
+    position left in the window still holds its own planes (the state is valid),
+    and the window is as long as the ring allows."""
+    L, R, H, d, W, kmax, Tmax, seq = 1, 3, 2, 4, 4, 2, 64, 0
+    rng = np.random.default_rng(5)
+    st = OR.OracleStore(L, R, H, d, W, Tmax, 1, kmax, np.float64)
+    K0, V0 = _block(rng, L, 12, R, H, d)
+    st.append([seq], [12], K0, V0)
+    st.evict([seq])
+    for _ in range(3):   # 3 * kmax = 6 speculative positions, ring capacity Wcap = 6
+        K, V = _block(rng, L, kmax, R, H, d)
+        st.append([seq], [kmax], K, V)
+        st.evict([seq])
+    st.truncate([seq], [12])
+    T, ws, rf = int(st.length[seq]), int(st.wstart[seq]), int(st.rfloor[seq])
+    assert T == 12 and rf == 12 and ws == 12   # every slot of 8..11 was overwritten
+    # A shorter rollback: positions 12..13 kept, 14..17 rejected.
+    st2 = OR.OracleStore(L, R, H, d, W, Tmax, 1, kmax, np.float64)
+    st2.append([seq], [12], K0, V0)
+    st2.evict([seq])
+    blocks = [_block(rng, L, kmax, R, H, d) for _ in range(3)]
+    for K, V in blocks:
+        st2.append([seq], [kmax], K, V)
+        st2.evict([seq])
+    st2.truncate([seq], [14])
+    T, ws = int(st2.length[seq]), int(st2.wstart[seq])
+    assert T == 14 and ws == 18 - st2.Wcap == 12   # positions 10, 11 overwritten by 16, 17
+    view = st2.plane_view(0, seq)
+    for i, p in enumerate(range(ws, T)):
+        t = p - 12
+        K, V = blocks[t // kmax]
+        assert np.array_equal(view["Kw"][:, :, i], np.swapaxes(K[0, 0, t % kmax, :R - 1], 0, 1))
+
+
+def test_rollback_past_window_start_and_noop():
+    L, R, H, d, W, kmax, seq = 1, 2, 1, 4, 3, 2, 0
+    rng = np.random.default_rng(6)
+    st = OR.OracleStore(L, R, H, d, W, 64, 1, kmax, np.float64)
+    K0, V0 = _block(rng, L, 10, R, H, d)
+    st.append([seq], [10], K0, V0)
+    st.evict([seq])
+    before = (int(st.length[seq]), int(st.wstart[seq]), int(st.rfloor[seq]))
+    st.truncate([seq], [10])
+    st.truncate([seq], [50])
+    assert (int(st.length[seq]), int(st.wstart[seq]), int(st.rfloor[seq])) == before
+    st.truncate([seq], [2])            # below the ring floor: empty window
+    assert (int(st.length[seq]), int(st.wstart[seq]), int(st.rfloor[seq])) == (2, 2, 2)
