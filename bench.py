@@ -169,7 +169,7 @@ def cpu_baseline(wl, budget_s=10.0):
     whole Huginn step in (layer, 11-head) blocks, repeated until about budget_s
     seconds of oracle time (input generation excluded)."""
     from oracle import oracle as OR
-    from tests.util import all_depth_rows, seq_planes
+    from depth_planed_kv_b200.synth_rows import all_depth_rows, seq_planes
     T, ws = wl.ctx, wl.ctx - wl.W
     br = S.all_depth_branches(1, wl.R, wl.k)
     blocks = []
@@ -228,7 +228,7 @@ def run_reference(args):
         return
     wl = S.huginn()
     from oracle import oracle as OR
-    from tests.util import all_depth_rows, seq_planes
+    from depth_planed_kv_b200.synth_rows import all_depth_rows, seq_planes
     T, ws = wl.ctx, wl.ctx - wl.W
     heads = np.arange(0, 4)
     br = S.all_depth_branches(1, wl.R, wl.k)
@@ -294,7 +294,7 @@ def main():
     from depth_planed_kv_b200 import build as B
     B.build()
     from depth_planed_kv_b200.ripe import RipeCache, launch_count
-    from tests.util import all_depth_rows
+    from depth_planed_kv_b200.synth_rows import all_depth_rows
 
     wl = S.huginn()
     nrep = 2

@@ -50,7 +50,7 @@ bool stream_capturing(cudaStream_t st) {
 namespace {
 
 struct Layout {
-    size_t kdeep, vdeep, kwin, vwin, len, ws, err, total;
+    size_t kdeep, vdeep, kwin, vwin, len, ws, rfloor, err, total;
 };
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -83,15 +83,21 @@ Layout layout_of(int L, int R, int H, int d, int W, int Tmax, int Bmax, int kmax
     y.vwin = y.kwin + ring;
     y.len = y.vwin + ring;
     y.ws = y.len + round256(sizeof(int32_t) * Bmax);
-    y.err = y.ws + round256(sizeof(int32_t) * Bmax);
+    y.rfloor = y.ws + round256(sizeof(int32_t) * Bmax);
+    y.err = y.rfloor + round256(sizeof(int32_t) * Bmax);
     y.total = y.err + 256;
     return y;
 }
 
 cudaStream_t as_stream(ripe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// A cache's store and scratch live on the device it was created on; every call
+// that enqueues work must find that device current.
 int check_cache(ripe_cache_t c) {
     if (!c) return fail(RIPE_ERR_INVALID_ARG, "cache is NULL");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device)
+        return fail(RIPE_ERR_INVALID_ARG, "the current device (%d) is not the cache's device (%d)", dev, c->device);
     return RIPE_OK;
 }
 
@@ -218,8 +224,16 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
     c->kdeep = c->base + y.kdeep; c->vdeep = c->base + y.vdeep;
     c->kwin = c->base + y.kwin; c->vwin = c->base + y.vwin;
     c->len = (int32_t*)(c->base + y.len); c->ws = (int32_t*)(c->base + y.ws);
+    c->rfloor = (int32_t*)(c->base + y.rfloor);
     c->err = (int32_t*)(c->base + y.err);
-    c->tc_ready = fused_supported(dtype, d) && make_tensor_maps(c) == 0;
+    c->tc_ready = false;
+    if (fused_supported(dtype, d)) {
+        const int tm = make_tensor_maps(c);
+        c->tc_ready = tm == 0;
+        if (!c->tc_ready)
+            fail(RIPE_OK, "tensor maps of this store cannot be built (code %d); verify uses the CUDA-core "
+                 "kernels (ripe_cache_verify_path reports 0)", tm);
+    }
     // Zeroed store: key tiles that overrun a region read finite values.
     cudaError_t e = cudaMemset(c->base, 0, y.total);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -233,8 +247,7 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
 }
 
 int ripe_cache_destroy(ripe_cache_t c) {
-    int rc = check_cache(c);
-    if (rc != RIPE_OK) return rc;
+    if (!c) return fail(RIPE_ERR_INVALID_ARG, "cache is NULL");
     cudaDeviceSynchronize();
     if (c->work) cudaFree(c->work);
     if (c->owns) cudaFree(c->base);
@@ -359,8 +372,16 @@ int ripe_synth_fill(ripe_cache_t c, const int32_t* seq_ids, const int32_t* T, in
     return RIPE_OK;
 }
 
+int ripe_cache_verify_path(ripe_cache_t c, int* path) {
+    int rc = check_cache(c);
+    if (rc != RIPE_OK) return rc;
+    if (!path) return fail(RIPE_ERR_INVALID_ARG, "path is NULL");
+    *path = c->tc_ready ? RIPE_PATH_FUSED_SM100 : RIPE_PATH_CUDA_CORE;
+    return RIPE_OK;
+}
+
 int ripe_cache_buffers(ripe_cache_t c, void** kdeep, void** vdeep, void** kwin, void** vwin, int32_t** len,
-                       int32_t** ws) {
+                       int32_t** ws, int32_t** rfloor) {
     int rc = check_cache(c);
     if (rc != RIPE_OK) return rc;
     if (kdeep) *kdeep = c->kdeep;
@@ -369,10 +390,12 @@ int ripe_cache_buffers(ripe_cache_t c, void** kdeep, void** vdeep, void** kwin, 
     if (vwin) *vwin = c->vwin;
     if (len) *len = c->len;
     if (ws) *ws = c->ws;
+    if (rfloor) *rfloor = c->rfloor;
     return RIPE_OK;
 }
 
-int ripe_read_meta(ripe_cache_t c, int32_t* len_host, int32_t* ws_host, ripe_stream_t stream) {
+int ripe_read_meta(ripe_cache_t c, int32_t* len_host, int32_t* ws_host, int32_t* rfloor_host,
+                   ripe_stream_t stream) {
     int rc = check_cache(c);
     if (rc != RIPE_OK) return rc;
     cudaStream_t st = as_stream(stream);
@@ -380,6 +403,8 @@ int ripe_read_meta(ripe_cache_t c, int32_t* len_host, int32_t* ws_host, ripe_str
     if (len_host) e = cudaMemcpyAsync(len_host, c->len, sizeof(int32_t) * c->Bmax, cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess && ws_host)
         e = cudaMemcpyAsync(ws_host, c->ws, sizeof(int32_t) * c->Bmax, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && rfloor_host)
+        e = cudaMemcpyAsync(rfloor_host, c->rfloor, sizeof(int32_t) * c->Bmax, cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "read_meta");
 }

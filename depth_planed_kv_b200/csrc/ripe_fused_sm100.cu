@@ -1059,16 +1059,15 @@ template <int D, int MT, int ST, int NW, int NS>
 cudaError_t launch_t(const TMaps& tm, const VerifyArgs& a, int gslots, bool pdl, cudaStream_t st) {
     using Lay = FusedLayout<D, MT, ST, NW, NS>;
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceOnce configured;
+    cudaError_t ce = per_device_once(configured, [] {
         cudaError_t e = cudaFuncSetAttribute(verify_kernel<D, MT, ST, NW, NS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(verify_kernel<D, MT, ST, NW, NS>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+        return cudaFuncSetAttribute(verify_kernel<D, MT, ST, NW, NS>,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    });
+    if (ce != cudaSuccess) return ce;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gslots, a.s.H, a.nsplit);
     cfg.blockDim = dim3(Lay::THREADS);

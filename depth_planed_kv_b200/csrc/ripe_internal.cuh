@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/ripe.h"
 
 struct ripe_cache_s {
@@ -15,7 +18,7 @@ struct ripe_cache_s {
     bool owns;
     char* base;
     char *kdeep, *vdeep, *kwin, *vwin;
-    int32_t *len, *ws, *err;
+    int32_t *len, *ws, *rfloor, *err;
     // Host-side upper bound of len over all sequences (grows with append/fill);
     // sizes the deep-region split grid without reading device metadata.
     int len_ub;
@@ -32,14 +35,16 @@ struct ripe_cache_s {
 // Store geometry, passed by value to kernels.
 struct StoreView {
     char *kdeep, *vdeep, *kwin, *vwin;
-    int32_t *len, *ws, *err;
+    // len: committed length; ws: window start; rfloor: lowest position whose ring
+    // slots still hold its own planes (ws >= rfloor; evict leaves it alone).
+    int32_t *len, *ws, *rfloor, *err;
     int L, R, H, d, Tmax, Bmax, Wcap, W, esize;
 };
 
 static inline StoreView store_view(const ripe_cache_s* c) {
     StoreView s;
     s.kdeep = c->kdeep; s.vdeep = c->vdeep; s.kwin = c->kwin; s.vwin = c->vwin;
-    s.len = c->len; s.ws = c->ws; s.err = c->err;
+    s.len = c->len; s.ws = c->ws; s.rfloor = c->rfloor; s.err = c->err;
     s.L = c->L; s.R = c->R; s.H = c->H; s.d = c->d; s.Tmax = c->Tmax; s.Bmax = c->Bmax;
     s.Wcap = c->Wcap; s.W = c->W; s.esize = c->esize;
     return s;
@@ -131,3 +136,27 @@ __host__ __device__ inline uint64_t synth_index(int layer, int plane, int seq, i
 
 // Kernel launch bookkeeping (counted on the host for every launch issued).
 void ripe_count_launch(int n = 1);
+
+// Per-device one-time set-up (kernel attributes such as the dynamic shared-memory
+// limit belong to a device): `fn` runs once for each device it is reached on,
+// with that device current; concurrent callers wait for the first.  A failed
+// set-up is retried on the next call.
+struct PerDeviceOnce {
+    std::atomic<uint64_t> done{0};  // one bit per device ordinal < 64
+    std::mutex mu;
+};
+
+template <typename F>
+inline cudaError_t per_device_once(PerDeviceOnce& once, F&& fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << dev;
+    if (once.done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(once.mu);
+    if (once.done.load(std::memory_order_relaxed) & bit) return cudaSuccess;
+    e = fn();
+    if (e == cudaSuccess) once.done.fetch_or(bit, std::memory_order_release);
+    return e;
+}

@@ -57,6 +57,11 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
                                         ripe_stream_t stream, size_t* scratch_needed) {
     if (scratch_needed) *scratch_needed = 0;
     if (!c) return ripe_fail(RIPE_ERR_INVALID_ARG, "cache is NULL");
+    // The static array's address is per device: the call must run on the cache's device.
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != c->device)
+        return ripe_fail(RIPE_ERR_INVALID_ARG, "the current device (%d) is not the cache's device (%d)", cur,
+                         c->device);
     if (layer < 0 || layer >= c->L || nbranch < 0 || nrows < 0)
         return ripe_fail(RIPE_ERR_INVALID_ARG, "layer, branch or row count out of range");
     if (nbranch == 0 || nrows == 0) return RIPE_OK;

@@ -64,7 +64,9 @@ __global__ void append_meta_kernel(StoreView s, const int32_t* __restrict__ seq_
     if (T + n > s.Tmax) { set_device_error(s.err, RIPE_DEVERR_CAPACITY); return; }
     const int nl = T + n;
     s.len[b] = nl;
+    // Positions below nl - Wcap no longer (or never) hold their planes in the ring.
     if (nl - s.Wcap > s.ws[b]) s.ws[b] = nl - s.Wcap;
+    if (nl - s.Wcap > s.rfloor[b]) s.rfloor[b] = nl - s.Wcap;
 }
 
 __global__ void evict_kernel(StoreView s, const int32_t* __restrict__ seq_ids, int nseq) {
@@ -83,8 +85,14 @@ __global__ void reset_kernel(StoreView s, const int32_t* __restrict__ seq_ids, i
     if (b < 0 || b >= s.Bmax) { set_device_error(s.err, RIPE_DEVERR_SEQ_RANGE); return; }
     s.len[b] = 0;
     s.ws[b] = 0;
+    s.rfloor[b] = 0;
 }
 
+// Rollback to the confirmed prefix (LoopSpec article, section on the second
+// branch): the state an evict at the confirmed length leaves, as far as the ring
+// still holds the planes -- positions pushed out of the window only by the
+// rejected tokens return to it.  len = min(len, T'), rfloor = min(rfloor, len),
+// ws = min(ws, max(len - W, rfloor)).  T' >= len changes nothing.
 __global__ void truncate_kernel(StoreView s, const int32_t* __restrict__ seq_ids,
                                 const int32_t* __restrict__ new_len, int nseq) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -95,8 +103,10 @@ __global__ void truncate_kernel(StoreView s, const int32_t* __restrict__ seq_ids
     const int t = new_len[i];
     if (t < 0) { set_device_error(s.err, RIPE_DEVERR_COUNT); return; }
     if (t < T) T = t;
+    const int rf = min(s.rfloor[b], T);
     s.len[b] = T;
-    if (s.ws[b] > T) s.ws[b] = T;
+    s.rfloor[b] = rf;
+    s.ws[b] = min(s.ws[b], max(T - s.W, rf));
 }
 
 struct Coefs { float c[64]; };
@@ -147,6 +157,7 @@ __global__ void synth_fill_kernel(StoreView s, int b, int T, uint64_t seed, Coef
 __global__ void set_meta_kernel(StoreView s, int b, int T) {
     s.len[b] = T;
     s.ws[b] = T - s.Wcap > 0 ? T - s.Wcap : 0;
+    s.rfloor[b] = s.ws[b];
 }
 
 }  // namespace

@@ -367,23 +367,22 @@ cudaError_t launch_seg(const VerifyArgs& a, int seg_first, int seg_count, int nb
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const SegShape g = seg_shape(a.s.d, (int)sizeof(Elem), keys_ub);
+    // The dynamic shared-memory limit is a per-device attribute of each instantiation.
+    auto configure = [](const void* fn) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        return cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared);
+    };
     if (a.s.d <= 64) {
-        static bool cfg = false;
-        if (!cfg) {
-            cudaFuncSetAttribute(seg_kernel<Elem, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-            cudaFuncSetAttribute(seg_kernel<Elem, 64>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-            cfg = true;
-        }
+        static PerDeviceOnce cfg;
+        cudaError_t e = per_device_once(cfg, [&] { return configure((const void*)seg_kernel<Elem, 64>); });
+        if (e != cudaSuccess) return e;
         seg_kernel<Elem, 64><<<(unsigned)grid, kWarps * 32, g.smem, st>>>(a, seg_first, seg_count, g.KT, g.ST);
     } else {
-        static bool cfg = false;
-        if (!cfg) {
-            cudaFuncSetAttribute(seg_kernel<Elem, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-            cudaFuncSetAttribute(seg_kernel<Elem, 128>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-            cfg = true;
-        }
+        static PerDeviceOnce cfg;
+        cudaError_t e = per_device_once(cfg, [&] { return configure((const void*)seg_kernel<Elem, 128>); });
+        if (e != cudaSuccess) return e;
         seg_kernel<Elem, 128><<<(unsigned)grid, kWarps * 32, g.smem, st>>>(a, seg_first, seg_count, g.KT, g.ST);
     }
     ripe_count_launch();

@@ -68,8 +68,9 @@ _sig("ripe_verify_attn_noalloc", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_f
                                   ctypes.POINTER(ctypes.c_size_t)])
 _sig("ripe_reserve_workspace", [_P, _I])
 _sig("ripe_synth_fill", [_P, _P, _P, _I, ctypes.c_uint64, _P, _P])
-_sig("ripe_cache_buffers", [_P] + [ctypes.POINTER(_P)] * 6)
-_sig("ripe_read_meta", [_P, _P, _P, _P])
+_sig("ripe_cache_verify_path", [_P, ctypes.POINTER(_I)])
+_sig("ripe_cache_buffers", [_P] + [ctypes.POINTER(_P)] * 7)
+_sig("ripe_read_meta", [_P, _P, _P, _P, _P])
 _sig("ripe_get_device_error", [_P, _P, _P])
 _sig("ripe_launch_count", [], ctypes.c_uint64)
 _sig("ripe_error_string", [_I], ctypes.c_char_p)
@@ -78,7 +79,7 @@ _sig("ripe_last_error", [], ctypes.c_char_p)
 EXPORTED = ["ripe_cache_bytes", "ripe_cache_create", "ripe_cache_destroy", "ripe_cache_reset",
             "ripe_append", "ripe_evict", "ripe_truncate", "ripe_verify_attn",
             "ripe_verify_attn_all_depths", "ripe_verify_attn_noalloc", "ripe_reserve_workspace",
-            "ripe_synth_fill",
+            "ripe_synth_fill", "ripe_cache_verify_path",
             "ripe_cache_buffers", "ripe_read_meta", "ripe_get_device_error", "ripe_launch_count",
             "ripe_error_string", "ripe_last_error"]
 
@@ -221,9 +222,15 @@ class RipeCache:
                                                 _stream(stream)), "ripe_verify_attn_all_depths")
 
     # --- inspection ------------------------------------------------------------
+    def ripe_cache_verify_path(self) -> int:
+        """1: the fused sm_100a kernel serves verify; 0: the CUDA-core kernels."""
+        out = ctypes.c_int()
+        _check(_lib.ripe_cache_verify_path(self.handle, ctypes.byref(out)), "ripe_cache_verify_path")
+        return out.value
+
     def buffers(self):
         """Torch views of the store parts (device memory owned by the cache)."""
-        ptrs = [ctypes.c_void_p() for _ in range(6)]
+        ptrs = [ctypes.c_void_p() for _ in range(7)]
         _check(_lib.ripe_cache_buffers(self.handle, *[ctypes.byref(p) for p in ptrs]), "ripe_cache_buffers")
         es = 2 if self.dtype == torch.bfloat16 else 4
         deep_shape = (self.layers, self.max_seqs, self.H, self.Tmax, self.d)
@@ -232,15 +239,18 @@ class RipeCache:
         return {"kdeep": mk(ptrs[0], deep_shape, self.dtype), "vdeep": mk(ptrs[1], deep_shape, self.dtype),
                 "kwin": mk(ptrs[2], ring_shape, self.dtype), "vwin": mk(ptrs[3], ring_shape, self.dtype),
                 "len": mk(ptrs[4], (self.max_seqs,), torch.int32),
-                "ws": mk(ptrs[5], (self.max_seqs,), torch.int32)}
+                "ws": mk(ptrs[5], (self.max_seqs,), torch.int32),
+                "rfloor": mk(ptrs[6], (self.max_seqs,), torch.int32)}
 
-    def ripe_read_meta(self, stream=None):
+    def ripe_read_meta(self, stream=None, with_rfloor=False):
+        """(len, ws) -- or (len, ws, rfloor) -- of every sequence, as host int32 arrays."""
         import numpy as np
         ln = np.zeros(self.max_seqs, np.int32)
         ws = np.zeros(self.max_seqs, np.int32)
-        _check(_lib.ripe_read_meta(self.handle, ln.ctypes.data_as(_P), ws.ctypes.data_as(_P), _stream(stream)),
-               "ripe_read_meta")
-        return ln, ws
+        rf = np.zeros(self.max_seqs, np.int32)
+        _check(_lib.ripe_read_meta(self.handle, ln.ctypes.data_as(_P), ws.ctypes.data_as(_P),
+                                   rf.ctypes.data_as(_P), _stream(stream)), "ripe_read_meta")
+        return (ln, ws, rf) if with_rfloor else (ln, ws)
 
     def ripe_get_device_error(self, stream=None) -> int:
         code = ctypes.c_int32()

@@ -24,6 +24,9 @@
  *     length above the committed length) skip the offending item and set the
  *     cache's device error word instead of trapping; read it with
  *     ripe_get_device_error().
+ *   - Every call that takes a cache must be made with the cache's device current
+ *     (the device that was current at ripe_cache_create); RIPE_ERR_INVALID_ARG
+ *     otherwise.  ripe_cache_destroy may be called from any device.
  *   - Pointers named *_dev are device pointers; *_host are host pointers.  The
  *     caller owns every buffer it passes; the library keeps no reference to
  *     them after the call's device work has run.
@@ -94,6 +97,9 @@ typedef struct {
  *                 position p lives in slot p mod Wcap, Wcap = W + kmax
  *   len[max_seqs], ws[max_seqs] (int32)                committed length T_b and
  *                 window start ws_b; positions ws_b <= p < T_b are live in the ring
+ *   rfloor[max_seqs] (int32)                           ring floor: the lowest position
+ *                 whose ring slots still hold its own planes (rfloor_b <= ws_b);
+ *                 append raises it like ws, evict does not
  * Memory per layer, sequence and head grows as T + W*(R-1) planes instead of R*T
  * (RIPE abstract, sentence on the 64-position window and 11.9% of the full
  * cache's memory).
@@ -118,7 +124,7 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
 /* Free the cache (and its store if the library allocated it).  Synchronises the device. */
 int ripe_cache_destroy(ripe_cache_t cache);
 
-/* Set len = ws = 0 for the listed sequences (device ids, nseq of them). */
+/* Set len = ws = rfloor = 0 for the listed sequences (device ids, nseq of them). */
 int ripe_cache_reset(ripe_cache_t cache, const int32_t* seq_ids_dev, int nseq,
                      ripe_stream_t stream);
 
@@ -153,8 +159,15 @@ int ripe_evict(ripe_cache_t cache, const int32_t* seq_ids_dev, int nseq, ripe_st
 /*
  * Roll the listed sequences back to a confirmed prefix (LoopSpec article,
  * section on the second branch: a rejected early draft discards the dependent
- * branch's work and decoding returns to the confirmed prefix):
- * len = min(len, new_len_dev[i]), ws = min(ws, len).
+ * branch's work and decoding returns to the confirmed prefix).  With
+ * T' = new_len_dev[i] >= 0 (device int32; a negative value skips the sequence
+ * and sets RIPE_DEVERR_COUNT):
+ *   len = min(len, T'),  rfloor = min(rfloor, len),  ws = min(ws, max(len - W, rfloor)).
+ * That is the state an evict at the confirmed length leaves: positions pushed out
+ * of the window only by the rejected tokens come back (their ring slots still
+ * hold every plane), as long as at most kmax positions are rolled back
+ * (Wcap = W + kmax).  Positions whose ring slots the rejected tokens overwrote
+ * stay at the deepest plane.  T' >= len changes nothing.
  */
 int ripe_truncate(ripe_cache_t cache, const int32_t* seq_ids_dev, const int32_t* new_len_dev,
                   int nseq, ripe_stream_t stream);
@@ -213,6 +226,8 @@ int ripe_verify_attn_all_depths(ripe_cache_t cache, int layer, const int32_t* se
  * ripe_verify_attn, but never allocates: its per-split partial results go to a
  * fixed device array of RIPE_NOALLOC_SCRATCH_BYTES owned by the library, which
  * every GPU that loads the library's device code holds until the process exits.
+ *   - The cache's device must be current (RIPE_ERR_INVALID_ARG otherwise), as for
+ *     every entry point that takes a cache.
  *   - The first call on each device looks up that array's device address
  *     (cudaGetSymbolAddress, with the device current); make that first call
  *     before any stream capture on the device.
@@ -247,12 +262,26 @@ int ripe_reserve_workspace(ripe_cache_t cache, int max_rows);
 int ripe_synth_fill(ripe_cache_t cache, const int32_t* seq_ids_host, const int32_t* T_host, int nseq,
                     uint64_t seed, const float* coef_host, ripe_stream_t stream);
 
-/* Device pointers of the store parts (tests compare them byte for byte). */
-int ripe_cache_buffers(ripe_cache_t cache, void** kdeep, void** vdeep, void** kwin, void** vwin,
-                       int32_t** len, int32_t** ws);
+/*
+ * Which kernels serve ripe_verify_attn* for this cache:
+ *   RIPE_PATH_FUSED_SM100 (1): the fused sm_100a kernel (tcgen05/TMEM deep plane,
+ *     TMA-fed, in-cluster merge) -- bf16 with d in {64, 96, 128};
+ *   RIPE_PATH_CUDA_CORE (0): the CUDA-core split and merge kernels (fp32, other head
+ *     sizes, or a store too large for the tensor maps -- ripe_cache_create then
+ *     leaves a note in ripe_last_error).
+ */
+enum { RIPE_PATH_CUDA_CORE = 0, RIPE_PATH_FUSED_SM100 = 1 };
+int ripe_cache_verify_path(ripe_cache_t cache, int* path);
 
-/* Copy len and ws of all max_seqs sequences to host arrays (synchronises stream). */
-int ripe_read_meta(ripe_cache_t cache, int32_t* len_host, int32_t* ws_host, ripe_stream_t stream);
+/* Device pointers of the store parts (tests compare them byte for byte); any
+ * output may be NULL. */
+int ripe_cache_buffers(ripe_cache_t cache, void** kdeep, void** vdeep, void** kwin, void** vwin,
+                       int32_t** len, int32_t** ws, int32_t** rfloor);
+
+/* Copy len, ws and rfloor of all max_seqs sequences to host arrays (each may be
+ * NULL; synchronises stream). */
+int ripe_read_meta(ripe_cache_t cache, int32_t* len_host, int32_t* ws_host, int32_t* rfloor_host,
+                   ripe_stream_t stream);
 
 /* Read and clear the device error word (synchronises stream). */
 int ripe_get_device_error(ripe_cache_t cache, int32_t* code_host, ripe_stream_t stream);

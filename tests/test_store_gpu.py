@@ -24,9 +24,10 @@ def compare_store(cache, model, what=""):
     for name, ref in (("kdeep", model.kdeep), ("vdeep", model.vdeep), ("kwin", model.kwin), ("vwin", model.vwin)):
         got = bits(buf[name])
         assert np.array_equal(got, ref), "%s: %s differs at %d elements" % (what, name, int((got != ref).sum()))
-    ln, ws = cache.ripe_read_meta()
+    ln, ws, rf = cache.ripe_read_meta(with_rfloor=True)
     assert np.array_equal(ln, model.length), (what, ln, model.length)
     assert np.array_equal(ws, model.wstart), (what, ws, model.wstart)
+    assert np.array_equal(rf, model.rfloor), (what, rf, model.rfloor)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -110,7 +111,7 @@ def test_synthetic_fill_equals_append_of_generator_planes(dtype, R, H, d, W, kma
                   torch.from_numpy(K).to(dtype).cuda(), torch.from_numpy(V).to(dtype).cuda())
     torch.cuda.synchronize()
     ba, bb = a.buffers(), b.buffers()
-    for name in ("kdeep", "vdeep", "kwin", "vwin", "len", "ws"):
+    for name in ("kdeep", "vdeep", "kwin", "vwin", "len", "ws", "rfloor"):
         assert np.array_equal(bits(ba[name]), bits(bb[name])), name
     a.close()
     b.close()

@@ -54,6 +54,35 @@ def test_noalloc_matches_allocating_entry_point_on_consecutive_calls(dtype):
     cache.close()
 
 
+def test_noalloc_halves_the_split_count_until_its_scratch_fits():
+    """A call whose first plan (8 deep splits: one sequence, two heads) needs more
+    than the fixed 32 MiB, but fits with fewer, longer splits: it runs with the
+    halved plan and matches the allocating entry point.  (Only the fused kernel's
+    plan can need this: the CUDA-core plan's split count already falls as the
+    rows grow.)"""
+    from depth_planed_kv_b200.ripe import branch_table
+    wl = S.Workload("noalloc_halve", 1, 4, 2, 64, 16, 141, 1, None, 0.88, 406, "bf16", 512, 141)
+    cache = make_cache(wl)
+    assert cache.ripe_cache_verify_path() == 1
+    fill(cache, wl, [300])
+    branches = [S.BranchSpec(0, 1 + i % 4, 141, i % 3, i % 2) for i in range(64)]   # 9024 rows
+    tb, nb, Q, Kb, Vb = _problem(wl, 0, branches, 1)
+    first_plan = Q.shape[0] * wl.H * 9 * (2 + wl.d) * 4     # 8 splits + the window partial
+    assert first_plan > 32 << 20
+    tol_abs, tol_rel = TOL["bf16"]
+    for _ in range(2):
+        ref = torch.full(Q.shape, float("nan"), dtype=Q.dtype, device="cuda")
+        cache.ripe_verify_attn(0, tb, nb, Q, Kb, Vb, ref)
+        got = torch.full_like(ref, float("nan"))
+        rc, used = cache.ripe_verify_attn_noalloc(0, tb, nb, Q, Kb, Vb, got)
+        torch.cuda.synchronize()
+        assert rc == 0 and used <= 32 << 20 and used < first_plan
+        a, r = errors(got.float().cpu().numpy(), ref.float().cpu().numpy())
+        assert a <= tol_abs and r <= tol_rel, (a, r)
+    assert cache.ripe_get_device_error() == 0
+    cache.close()
+
+
 def test_noalloc_refuses_calls_beyond_its_fixed_scratch():
     from depth_planed_kv_b200.ripe import RIPE_ERR_CAPACITY, branch_table
     wl = S.Workload("noalloc_big", 1, 4, 32, 128, 8, 64, 1, 64, 0.88, 5, "bf16", 128, 64)
