@@ -45,6 +45,9 @@ def _load():
                                                                      P, P, P, ctypes.c_double,
                                                                      ctypes.c_int, P, P]
         lib.oracle_verify.restype = ctypes.c_int
+        lib.oracle_verify_sliding.argtypes = [ctypes.c_int] * 5 + [P] * 8 + [ctypes.c_int, P, ctypes.c_int,
+                                                                             P, P, P, ctypes.c_double, P, P]
+        lib.oracle_verify_sliding.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -56,6 +59,66 @@ def num_threads() -> int:
 
 def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _pack(seqs, Q, Kb, Vb):
+    """The flat arrays oracle_verify* take: per-sequence views concatenated."""
+    Q = np.ascontiguousarray(Q, dtype=np.float64)
+    Kb = np.ascontiguousarray(Kb, dtype=np.float64)
+    Vb = np.ascontiguousarray(Vb, dtype=np.float64)
+    nrows, H, d = Q.shape
+    R = None
+    deep_k, deep_v, win_k, win_v, deep_off, win_off = [], [], [], [], [], []
+    dpos = wpos = 0
+    for s in seqs:
+        T, ws = int(s["T"]), int(s["ws"])
+        lo = min(ws, T)
+        kd = np.ascontiguousarray(s["Kd"], dtype=np.float64)
+        assert kd.shape == (H, T, d), (kd.shape, (H, T, d))
+        deep_k.append(kd.ravel()); deep_v.append(np.ascontiguousarray(s["Vd"], dtype=np.float64).ravel())
+        deep_off.append(dpos); dpos += kd.size
+        kw = s.get("Kw")
+        if kw is not None and kw.size:
+            kw = np.ascontiguousarray(kw, dtype=np.float64)
+            assert kw.shape[0] == H and kw.shape[2] == T - lo and kw.shape[3] == d
+            R = kw.shape[1] + 1 if R is None else R
+            win_k.append(kw.ravel()); win_v.append(np.ascontiguousarray(s["Vw"], dtype=np.float64).ravel())
+            win_off.append(wpos); wpos += kw.size
+        else:
+            win_off.append(wpos)
+    R = int(seqs[0]["R"]) if R is None else R
+    for s in seqs:
+        assert int(s.get("R", R)) == R
+    cat = lambda xs: np.concatenate(xs) if xs else np.zeros(1)
+    return dict(Q=Q, Kb=Kb, Vb=Vb, H=H, d=d, R=R, nrows=nrows,
+                Kd=cat(deep_k), Vd=cat(deep_v), Kw=cat(win_k), Vw=cat(win_v),
+                T=np.array([int(s["T"]) for s in seqs], dtype=np.int64),
+                ws=np.array([int(s["ws"]) for s in seqs], dtype=np.int64),
+                do=np.array(deep_off, dtype=np.int64), wo=np.array(win_off, dtype=np.int64))
+
+
+def verify_sliding(seqs: Sequence[Dict], branches: np.ndarray, Q: np.ndarray, Kb: np.ndarray,
+                   Vb: np.ndarray, W: int, scale: float):
+    """Verify-attention under the per-query sliding-window reading (the RIPE
+    abstract's fifth sentence read per query): draft token j at position T + j sees
+    positions T+j-W+1 .. T+j at its own depth r -- committed positions among them
+    only if the store still holds their planes (p >= ws) -- and everything older at
+    the deepest plane R; an older draft token's plane R is its depth-R row.
+    ``branches`` must be the all-depths form (row0 = s*k*R + r - 1, row_stride R).
+    Same inputs and outputs as ``verify`` otherwise; the definition is evaluated
+    directly (all scores of a row, one softmax)."""
+    lib = _load()
+    a = _pack(seqs, Q, Kb, Vb)
+    br = np.ascontiguousarray(branches, dtype=np.int32).reshape(-1, 5)
+    O = np.zeros((a["nrows"], a["H"], a["d"]), dtype=np.float64)
+    lse = np.zeros((a["nrows"], a["H"]), dtype=np.float64)
+    rc = lib.oracle_verify_sliding(len(seqs), a["H"], a["d"], a["R"], int(W), _ptr(a["T"]), _ptr(a["ws"]),
+                                   _ptr(a["do"]), _ptr(a["Kd"]), _ptr(a["Vd"]), _ptr(a["wo"]), _ptr(a["Kw"]),
+                                   _ptr(a["Vw"]), br.shape[0], _ptr(br), a["nrows"], _ptr(a["Q"]), _ptr(a["Kb"]),
+                                   _ptr(a["Vb"]), float(scale), _ptr(O), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_verify_sliding rejected its arguments (code %d)" % rc)
+    return O, lse
 
 
 def verify(seqs: Sequence[Dict], branches: np.ndarray, Q: np.ndarray, Kb: np.ndarray,

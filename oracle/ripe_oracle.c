@@ -236,3 +236,97 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/*
+ * Sliding-window reading (the RIPE abstract's fifth sentence, read per query):
+ * the query of draft token j sits at position T + j and sees the W most recent
+ * positions T+j-W+1 .. T+j at its own depth r, everything older at the deepest
+ * plane R.  Committed position p is read at plane r if p >= T + j - W + 1 and the
+ * store still holds its planes (p >= ws), else at plane R; draft token j' <= j at
+ * plane r if j' >= j - W + 1, else at plane R.  The plane-R key and value of draft
+ * token j' are those of the same token's depth-R row, so the branches must be the
+ * all-depths form of one sequence each: branch (s, r) has row0 = s*k*R + r - 1 and
+ * row_stride R.  Every score of a row is gathered, then one max-subtracted softmax
+ * (the definition written out, as mode 0).
+ */
+int oracle_verify_sliding(int nseq, int H, int d, int R, int W,
+                          const int64_t* T, const int64_t* ws,
+                          const int64_t* deep_off, const double* Kd, const double* Vd,
+                          const int64_t* win_off, const double* Kw, const double* Vw,
+                          int nbranch, const int32_t* branches,
+                          int nrows, const double* Q, const double* Kb, const double* Vb,
+                          double scale, double* O, double* lse) {
+    if (nseq < 0 || H <= 0 || d <= 0 || R <= 0 || W < 0 || nbranch < 0 || nrows < 0) return 1;
+    seq_view* seqs = (seq_view*)calloc(nseq > 0 ? nseq : 1, sizeof(seq_view));
+    if (!seqs) return 2;
+    int64_t maxT = 0;
+    for (int b = 0; b < nseq; ++b) {
+        seqs[b].T = T[b];
+        seqs[b].ws = ws[b];
+        seqs[b].lo = ws[b] < T[b] ? ws[b] : T[b];
+        seqs[b].kd = Kd + deep_off[b];
+        seqs[b].vd = Vd + deep_off[b];
+        seqs[b].kw = Kw ? Kw + win_off[b] : NULL;
+        seqs[b].vw = Vw ? Vw + win_off[b] : NULL;
+        if (T[b] > maxT) maxT = T[b];
+    }
+    int maxn = 0;
+    for (int i = 0; i < nbranch; ++i) {
+        const int32_t* b = branches + 5 * i;
+        if (b[0] < 0 || b[0] >= nseq || b[1] < 1 || b[1] > R || b[2] < 0 || b[4] != R) { free(seqs); return 1; }
+        if (b[2] > maxn) maxn = b[2];
+        const int64_t rowR0 = (int64_t)b[3] - (b[1] - 1) + (R - 1);
+        if (b[2] > 0 && (b[3] < 0 || rowR0 + (int64_t)(b[2] - 1) * R >= nrows)) { free(seqs); return 1; }
+    }
+    problem P = {H, d, R, seqs, branches, Q, Kb, Vb, scale};
+    int64_t nunits = (int64_t)nbranch * H;
+#pragma omp parallel
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)(maxT + maxn + 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t u = 0; u < nunits; ++u) {
+            const int i = (int)(u / H), h = (int)(u % H);
+            const int32_t* b = branches + 5 * i;
+            const seq_view* s = seqs + b[0];
+            const int r = b[1], row0 = b[3];
+            const int64_t rowR0 = (int64_t)row0 - (r - 1) + (R - 1);
+            for (int j = 0; j < b[2]; ++j) {
+                const int64_t row = row0 + (int64_t)j * R;
+                const double* q = Q + (row * H + h) * d;
+                const int64_t start = s->T + j - W + 1;   /* first position of the row's window */
+                int64_t n = 0;
+                for (int64_t p = 0; p < s->T; ++p) {
+                    const int plane = (p >= start && p >= s->ws) ? r : R;
+                    scores[n++] = scale * dot(q, committed_row(&P, s, h, p, plane, 0), d);
+                }
+                for (int jj = 0; jj <= j; ++jj) {
+                    const int64_t kr = (jj >= j - W + 1) ? row0 + (int64_t)jj * R : rowR0 + (int64_t)jj * R;
+                    scores[n++] = scale * dot(q, Kb + (kr * H + h) * d, d);
+                }
+                double m = -INFINITY;
+                for (int64_t t = 0; t < n; ++t) m = scores[t] > m ? scores[t] : m;
+                double sum = 0.0;
+                for (int64_t t = 0; t < n; ++t) { scores[t] = exp(scores[t] - m); sum += scores[t]; }
+                double* out = O + (row * H + h) * d;
+                for (int c = 0; c < d; ++c) out[c] = 0.0;
+                n = 0;
+                for (int64_t p = 0; p < s->T; ++p) {
+                    const int plane = (p >= start && p >= s->ws) ? r : R;
+                    const double* v = committed_row(&P, s, h, p, plane, 1);
+                    const double w = scores[n++] / sum;
+                    for (int c = 0; c < d; ++c) out[c] += w * v[c];
+                }
+                for (int jj = 0; jj <= j; ++jj) {
+                    const int64_t kr = (jj >= j - W + 1) ? row0 + (int64_t)jj * R : rowR0 + (int64_t)jj * R;
+                    const double* v = Vb + (kr * H + h) * d;
+                    const double w = scores[n++] / sum;
+                    for (int c = 0; c < d; ++c) out[c] += w * v[c];
+                }
+                lse[row * H + h] = m + log(sum);
+            }
+        }
+        free(scores);
+    }
+    free(seqs);
+    return 0;
+}

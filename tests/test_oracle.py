@@ -410,3 +410,91 @@ def test_rollback_past_window_start_and_noop():
     assert (int(st.length[seq]), int(st.wstart[seq]), int(st.rfloor[seq])) == before
     st.truncate([seq], [2])            # below the ring floor: empty window
     assert (int(st.length[seq]), int(st.wstart[seq]), int(st.rfloor[seq])) == (2, 2, 2)
+
+
+# --- the sliding-window reading (the RIPE abstract's fifth sentence, per query) -----
+
+def _sliding(wl, T, ws, k, W, seq=3, layer=0):
+    views = [seq_planes(wl, layer, seq, T, ws)]
+    table, Q, Kb, Vb = all_depth_rows(wl, layer, 1, [seq], k)
+    O, lse = OR.verify_sliding(views, table, Q, Kb, Vb, W, 1 / math.sqrt(wl.d))
+    return O, lse, (views, table, Q, Kb, Vb)
+
+
+def test_sliding_window_covering_everything_is_full_cache():
+    wl = small(R=4, H=2, d=8)
+    T, k = 20, 3
+    O, _, (views, table, Q, Kb, Vb) = _sliding(wl, T, 0, k, W=T + k + 5)
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            for h in range(wl.H):
+                keys = list(kf[h, r - 1]) + [Kb[row0 + jj * stride, h] for jj in range(j + 1)]
+                vals = list(vf[h, r - 1]) + [Vb[row0 + jj * stride, h] for jj in range(j + 1)]
+                assert np.abs(O[row, h] - sdpa_row(Q[row, h], keys, vals, scale)).max() <= 1e-13
+
+
+def test_sliding_zero_window_reads_the_deepest_plane_only():
+    """W = 0: every committed position and every draft token, the query's own
+    included, at plane R (a draft token's plane R is its depth-R row)."""
+    wl = small(R=4, H=2, d=8)
+    T, k = 20, 3
+    R = wl.R
+    O, _, (views, table, Q, Kb, Vb) = _sliding(wl, T, T, k, W=0)
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            for h in range(wl.H):
+                keys = list(kf[h, R - 1]) + [Kb[jj * R + R - 1, h] for jj in range(j + 1)]
+                vals = list(vf[h, R - 1]) + [Vb[jj * R + R - 1, h] for jj in range(j + 1)]
+                assert np.abs(O[row, h] - sdpa_row(Q[row, h], keys, vals, scale)).max() <= 1e-13
+
+
+def test_sliding_pure_python_brute_force():
+    wl = small(R=3, H=1, d=4, W=2, k=3, seed=11)
+    T, ws, k, W, R = 6, 3, 3, 2, 3
+    O, lse, (views, table, Q, Kb, Vb) = _sliding(wl, T, ws, k, W)
+    kf, vf = full_planes(wl, 0, 3, T)
+    scale = 1 / math.sqrt(wl.d)
+    for (seq, r, n, row0, stride) in table:
+        for j in range(n):
+            row = row0 + j * stride
+            q = [float(x) for x in Q[row, 0]]
+            keys, vals = [], []
+            for p in range(T):
+                plane = r if (p >= T + j - W + 1 and p >= ws) else R
+                keys.append([float(x) for x in kf[0, plane - 1, p]])
+                vals.append([float(x) for x in vf[0, plane - 1, p]])
+            for jj in range(j + 1):
+                src = row0 + jj * stride if jj >= j - W + 1 else jj * R + R - 1
+                keys.append([float(x) for x in Kb[src, 0]])
+                vals.append([float(x) for x in Vb[src, 0]])
+            s = [scale * sum(a * b for a, b in zip(q, kk)) for kk in keys]
+            e = [math.exp(x) for x in s]
+            z = sum(e)
+            o = [sum(e[t] * vals[t][c] for t in range(len(e))) / z for c in range(wl.d)]
+            assert max(abs(O[row, 0, c] - o[c]) for c in range(wl.d)) < 1e-12
+            assert abs(lse[row, 0] - math.log(z)) < 1e-12
+
+
+@pytest.mark.parametrize("W,k", [(4, 4), (6, 4), (3, 4), (1, 4)])
+def test_sliding_block_independence_iff_window_covers_block(W, k):
+    """BI4 as a computation: the depth-R rows' block planes reach a depth-r < R row
+    only through draft tokens read at plane R, which happens iff W < k."""
+    wl = small(R=4, H=2, d=8, W=W, k=k)
+    T, R = 20, wl.R
+    O, _, (views, table, Q, Kb, Vb) = _sliding(wl, T, T - W, k, W)
+    Kp, Vp = Kb.copy(), Vb.copy()
+    rng = np.random.default_rng(2)
+    for j in range(k):
+        Kp[j * R + R - 1] += rng.standard_normal(Kp[0].shape).astype(np.float32)
+        Vp[j * R + R - 1] += rng.standard_normal(Vp[0].shape).astype(np.float32)
+    O2, _ = OR.verify_sliding(views, table, Q, Kp, Vp, W, 1 / math.sqrt(wl.d))
+    shallow = [j * R + r - 1 for j in range(k) for r in range(1, R)]
+    changed = not np.array_equal(O[shallow], O2[shallow])
+    assert changed == (W < k)
+    assert changed == bool(OR.sliding_block_reads_deepest(W, k).any())
