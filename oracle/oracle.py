@@ -240,7 +240,19 @@ class OracleStore:
     window forward come back into the window; positions whose ring slots the
     rejected tokens overwrote cannot (with Wcap = W + kmax that happens only when
     more than kmax positions are rolled back).  A truncate to T' >= T_b changes
-    nothing.
+    nothing.  A fork cannot be truncated below its fork position (flagged,
+    skipped): release it instead.
+
+    Branch forks (LoopSpec article, section on deployment: a KV cache per branch,
+    rejected continuations deleted).  fork(parent p -> child c) gives slot c the
+    parent's state without copying its deep prefix: base[c] = p and fpos[c] =
+    floor64(T_p) (a multiple of 64, the deep tile), so positions below fpos[c] are
+    read from p's deep plane; the child gets its own copies of p's deep rows
+    fpos..T_p-1 and of p's whole ring, and its own len/ws/rfloor.  Appends to c
+    then write c's own rows.  While c lives, p must keep its deep rows below
+    fpos[c] (no truncate below it).  Only a sequence that is not itself a fork can
+    be forked (else flagged, skipped).  release(c) frees the slot: len = ws =
+    rfloor = 0, base = itself, fpos = 0.
     """
 
     def __init__(self, L, R, H, d, W, Tmax, Bmax, kmax, np_dtype):
@@ -254,13 +266,36 @@ class OracleStore:
         self.length = np.zeros(Bmax, dtype=np.int32)
         self.wstart = np.zeros(Bmax, dtype=np.int32)
         self.rfloor = np.zeros(Bmax, dtype=np.int32)
+        self.base = np.arange(Bmax, dtype=np.int32)
+        self.fpos = np.zeros(Bmax, dtype=np.int32)
         self.flagged = False
 
     def reset(self, seq_ids):
+        """Empty the listed slots (a fork is released: it no longer reads its parent)."""
         for b in seq_ids:
             self.length[b] = 0
             self.wstart[b] = 0
             self.rfloor[b] = 0
+            self.base[b] = b
+            self.fpos[b] = 0
+
+    def fork(self, parent_ids, child_ids):
+        for p, c in zip(parent_ids, child_ids):
+            p, c = int(p), int(c)
+            if not (0 <= p < self.Bmax and 0 <= c < self.Bmax) or p == c or self.base[p] != p:
+                self.flagged = True
+                continue
+            T = int(self.length[p])
+            f = T // 64 * 64
+            self.kdeep[:, c, :, f:T] = self.kdeep[:, p, :, f:T]
+            self.vdeep[:, c, :, f:T] = self.vdeep[:, p, :, f:T]
+            self.kwin[:, c] = self.kwin[:, p]
+            self.vwin[:, c] = self.vwin[:, p]
+            self.length[c] = T
+            self.wstart[c] = self.wstart[p]
+            self.rfloor[c] = self.rfloor[p]
+            self.base[c] = p
+            self.fpos[c] = f
 
     def append(self, seq_ids, n_acc, K, V):
         """K, V: [L][nseq][kmax_in][R][H][d]; plane index r-1 along axis 3."""
@@ -290,7 +325,7 @@ class OracleStore:
 
     def truncate(self, seq_ids, new_len):
         for i, b in enumerate(seq_ids):
-            if int(new_len[i]) < 0:
+            if int(new_len[i]) < 0 or (self.base[b] != b and int(new_len[i]) < int(self.fpos[b])):
                 self.flagged = True
                 continue
             T = min(int(self.length[b]), int(new_len[i]))
@@ -300,14 +335,17 @@ class OracleStore:
             self.wstart[b] = min(int(self.wstart[b]), max(T - self.W, rf))
 
     def plane_view(self, layer: int, b: int):
-        """What a verify reads for sequence b: the oracle's logical input dict."""
+        """What a verify reads for sequence b: the oracle's logical input dict (a
+        fork's deep positions below its fork position come from its parent)."""
         T, ws = int(self.length[b]), int(self.wstart[b])
         lo = min(ws, T)
         pos = np.arange(lo, T)
         slots = pos % self.Wcap
+        f, base = min(int(self.fpos[b]), T), int(self.base[b])
+        kd = np.concatenate([self.kdeep[layer, base, :, :f, :], self.kdeep[layer, b, :, f:T, :]], axis=1)
+        vd = np.concatenate([self.vdeep[layer, base, :, :f, :], self.vdeep[layer, b, :, f:T, :]], axis=1)
         return {
-            "T": T, "ws": ws, "R": self.R,
-            "Kd": self.kdeep[layer, b, :, :T, :], "Vd": self.vdeep[layer, b, :, :T, :],
+            "T": T, "ws": ws, "R": self.R, "Kd": kd, "Vd": vd,
             "Kw": self.kwin[layer, b][:, :, slots, :], "Vw": self.vwin[layer, b][:, :, slots, :],
         }
 

@@ -498,3 +498,61 @@ def test_sliding_block_independence_iff_window_covers_block(W, k):
     changed = not np.array_equal(O[shallow], O2[shallow])
     assert changed == (W < k)
     assert changed == bool(OR.sliding_block_reads_deepest(W, k).any())
+
+
+# --- branch forks (LoopSpec article, deployment section: a KV cache per branch) -----
+
+@pytest.mark.parametrize("T0,W,kmax", [(130, 8, 4), (64, 16, 8), (5, 4, 4), (200, 0, 3)])
+def test_fork_equals_a_store_that_appended_the_branch(T0, W, kmax):
+    """A fork that appends its branch's tokens reads exactly what a store that
+    appended the parent's tokens and then the branch's would read; the parent is
+    untouched; releasing the fork empties it."""
+    L, R, H, d, Tmax, B = 1, 4, 2, 8, 400, 4
+    rng = np.random.default_rng(T0 + W)
+    st = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np.float64)
+    ref = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np.float64)
+    K0, V0 = _block(rng, L, T0, R, H, d)
+    for s in (st, ref):
+        s.append([0], [T0], K0, V0)
+        s.evict([0])
+    parent_before = {k: v.copy() for k, v in st.plane_view(0, 0).items() if isinstance(v, np.ndarray)}
+    st.fork([0], [2])
+    assert not st.flagged
+    for step in range(3):
+        n = int(rng.integers(1, kmax + 1))
+        K, V = _block(rng, L, n, R, H, d)
+        st.append([2], [n], K, V)
+        st.evict([2])
+        ref.append([0], [n], K, V)
+        ref.evict([0])
+        vs, vr = st.plane_view(0, 2), ref.plane_view(0, 0)
+        assert vs["T"] == vr["T"] and vs["ws"] == vr["ws"]
+        for key in ("Kd", "Vd", "Kw", "Vw"):
+            assert np.array_equal(vs[key], vr[key]), (step, key)
+        s1 = int(rng.integers(0, 2 ** 31))
+        Os, _ = _all_depth_verify(st, 2, np.random.default_rng(s1), R, H, d)
+        Or, _ = _all_depth_verify(ref, 0, np.random.default_rng(s1), R, H, d)
+        assert np.array_equal(Os[:], Or[:])
+    after = st.plane_view(0, 0)
+    for k, v in parent_before.items():
+        assert np.array_equal(after[k], v)
+    st.reset([2])
+    assert st.length[2] == 0 and st.base[2] == 2 and st.fpos[2] == 0
+
+
+def test_fork_rules():
+    L, R, H, d = 1, 3, 1, 4
+    st = OR.OracleStore(L, R, H, d, 4, 300, 4, 4, np.float64)
+    rng = np.random.default_rng(9)
+    K0, V0 = _block(rng, L, 150, R, H, d)
+    st.append([0], [150], K0, V0)
+    st.fork([0], [1])
+    assert not st.flagged and st.fpos[1] == 128 and st.base[1] == 0
+    st.fork([1], [2])                  # a fork of a fork
+    assert st.flagged
+    st.flagged = False
+    st.truncate([1], [100])            # below the fork position
+    assert st.flagged and st.length[1] == 150
+    st.flagged = False
+    st.truncate([1], [140])            # above it: an ordinary rollback
+    assert not st.flagged and st.length[1] == 140
