@@ -124,6 +124,13 @@ int ensure_workspace(ripe_cache_s* c, size_t need, cudaStream_t st) {
         cudaGetLastError();
         return fail(RIPE_ERR_OOM, "cudaMalloc(%zu) for verify scratch failed", sz);
     }
+    // The slice counters at its start must be zero (each call leaves them so).
+    cudaError_t e = cudaMemset(p, 0, sz);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(e, "zeroing the verify scratch");
+    }
     c->work = p;
     c->work_bytes = sz;
     return RIPE_OK;
@@ -143,9 +150,13 @@ int verify_common(ripe_cache_s* c, int layer, const BranchArgs& ba, const void* 
     // A captured launch replays while the sequences grow: its plan covers Tmax.
     const VerifyPlan plan = plan_verify(c, ba.nbranch, ba.nrows, ba.max_ntok, ba.table == nullptr,
                                         stream_capturing(st));
+    if (ba.sliding && !plan.persist)
+        return fail(RIPE_ERR_UNSUPPORTED, "the sliding window needs the persistent sm_100a kernel (bf16, d in "
+                    "{64,96,128}, k*R <= 256, R*ceil(k/8) <= %d)", kPersistSlices);
     int rc = ensure_workspace(c, plan.work_bytes, st);
     if (rc != RIPE_OK) return rc;
-    cudaError_t e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, c->work, st);
+    cudaError_t e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, c->work,
+                                  static_cast<char*>(c->work) + counter_bytes(c), st);
     if (e != cudaSuccess) return cuda_fail(e, "verify launch");
     return RIPE_OK;
 }
@@ -340,6 +351,25 @@ int ripe_verify_attn_all_depths(ripe_cache_t c, int layer, const int32_t* seq_id
     return verify_common(c, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, as_stream(stream));
 }
 
+int ripe_verify_attn_all_depths_sliding(ripe_cache_t c, int layer, const int32_t* seq_ids, int nseq, int k,
+                                        const void* Q, const void* Kb, const void* Vb, const int32_t* ctx,
+                                        float scale, void* O, float* lse, ripe_stream_t stream) {
+    int rc = check_cache(c);
+    if (rc != RIPE_OK) return rc;
+    if (nseq < 0 || nseq > c->Bmax) return fail(RIPE_ERR_INVALID_ARG, "nseq=%d outside [0,%d]", nseq, c->Bmax);
+    if (k < 1 || k > 4096) return fail(RIPE_ERR_INVALID_ARG, "k=%d outside [1,4096]", k);
+    if (nseq > 0 && !seq_ids) return fail(RIPE_ERR_INVALID_ARG, "seq_ids is NULL");
+    BranchArgs ba{};
+    ba.table = nullptr;
+    ba.seq_ids = seq_ids;
+    ba.nbranch = nseq * c->R;
+    ba.nrows = nseq * k * c->R;
+    ba.k = k;
+    ba.max_ntok = k;
+    ba.sliding = 1;
+    return verify_common(c, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, as_stream(stream));
+}
+
 int ripe_reserve_workspace(ripe_cache_t c, int max_rows) {
     int rc = check_cache(c);
     if (rc != RIPE_OK) return rc;
@@ -369,6 +399,34 @@ int ripe_synth_fill(ripe_cache_t c, const int32_t* seq_ids, const int32_t* T, in
         if (e != cudaSuccess) return cuda_fail(e, "synthetic fill launch");
         if (T[i] > c->len_ub) c->len_ub = T[i];
     }
+    return RIPE_OK;
+}
+
+int ripe_accept(int nseq, int k, int V, const float* zp, const float* zq, const float* zf, const int32_t* x1,
+                const int32_t* x2, const float* u, float temperature, int32_t* n_accepted, int32_t* token,
+                int32_t* path, ripe_stream_t stream) {
+    if (nseq < 0 || nseq > (1 << 20)) return fail(RIPE_ERR_INVALID_ARG, "nseq=%d outside [0, 2^20]", nseq);
+    if (k < 1 || k > 4096) return fail(RIPE_ERR_INVALID_ARG, "k=%d outside [1, 4096]", k);
+    if (V < 1 || V > (1 << 24)) return fail(RIPE_ERR_INVALID_ARG, "V=%d outside [1, 2^24]", V);
+    if (!(temperature >= 0.f) || isinf(temperature))
+        return fail(RIPE_ERR_INVALID_ARG, "temperature must be finite and >= 0");
+    if (nseq == 0) return RIPE_OK;
+    if (!zp || !zq || !x1 || !u || !n_accepted || !token || !path || (zf && !x2))
+        return fail(RIPE_ERR_INVALID_ARG, "NULL pointer argument (x2 is required with zf)");
+    const auto mis = [](const void* p) { return ((uintptr_t)p & 3u) != 0; };
+    if (mis(zp) || mis(zq) || (zf && mis(zf)) || mis(x1) || (x2 && mis(x2)) || mis(u) || mis(n_accepted) ||
+        mis(token) || mis(path))
+        return fail(RIPE_ERR_UNALIGNED, "arrays must be 4-byte aligned");
+    cudaError_t e = launch_accept(nseq, k, V, zp, zq, zf, x1, x2, u, temperature, n_accepted, token, path,
+                                  as_stream(stream));
+    return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "accept launch");
+}
+
+int ripe_debug_stall_next_verify(ripe_cache_t c, long long cycles) {
+    int rc = check_cache(c);
+    if (rc != RIPE_OK) return rc;
+    if (cycles < 0 || cycles > (1ll << 31)) return fail(RIPE_ERR_INVALID_ARG, "cycles=%lld outside [0, 2^31]", cycles);
+    c->probe_cycles.store(cycles);
     return RIPE_OK;
 }
 
@@ -417,6 +475,12 @@ int ripe_get_device_error(ripe_cache_t c, int32_t* code_host, ripe_stream_t stre
     cudaError_t e = cudaMemcpyAsync(code_host, c->err, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(c->err, 0, sizeof(int32_t), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    // A kernel that gave up a wait may have left slice counters mid-count: zero
+    // them so that later calls merge correctly.
+    if (e == cudaSuccess && *code_host == RIPE_DEVERR_TIMEOUT && c->work) {
+        e = cudaMemsetAsync(c->work, 0, counter_bytes(c), st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
     return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "get_device_error");
 }
 

@@ -1115,24 +1115,27 @@ static EncodeFn encode_fn() {
 
 bool fused_supported(int dtype, int d) { return dtype == RIPE_BF16 && (d == 64 || d == 96 || d == 128); }
 
+// This call's Q viewed as [rows][H][d]: boxes of 128 rows x 32 columns of one head
+// (the stacked-query tile of the deep region).
+bool make_q_map(void* tmap, const VerifyArgs& a) {
+    const EncodeFn encode = encode_fn();
+    if (!encode) return false;
+    const int d = a.s.d;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)a.s.H, (cuuint64_t)a.ba.nrows};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)a.s.H * d * 2};
+    const cuuint32_t box[3] = {32, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode(reinterpret_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<char*>(a.Q),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_fused(const void* tmaps, const VerifyArgs& args, int gslots, int mt, bool pdl, cudaStream_t st) {
-    // The cache's maps plus one of this call's Q, viewed as [rows][H][d]: boxes of
-    // 128 rows x 32 columns of one head (the stacked-query tile of the deep region).
+    // The cache's first six maps plus one of this call's Q.
     TMaps tm;
     memcpy(&tm, tmaps, 6 * sizeof(CUtensorMap));
     VerifyArgs a = args;
-    a.q_tma = 0;
-    if (const EncodeFn encode = encode_fn()) {
-        const int d = a.s.d;
-        const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)a.s.H, (cuuint64_t)a.ba.nrows};
-        const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)a.s.H * d * 2};
-        const cuuint32_t box[3] = {32, 1, 128};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        if (encode(&tm.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<char*>(a.Q), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
-            a.q_tma = 1;
-    }
+    a.q_tma = make_q_map(&tm.q, a) ? 1 : 0;
     const int d = a.s.d;
     // <D, M tiles, deep stages, window warps, window stages>, each within 227 KB of shared memory.
     if (mt == 1) {
@@ -1148,14 +1151,15 @@ cudaError_t launch_fused(const void* tmaps, const VerifyArgs& args, int gslots, 
 }
 
 // Tensor maps: 2-D [rows][d] bf16 views, 32-column boxes with the 64-byte swizzle
-// the kernel's shared-memory layouts expect.  Deep planes (rows = L*Bmax*H*Tmax)
+// the kernels' shared-memory layouts expect.  Deep planes (rows = L*Bmax*H*Tmax)
 // in 64-row boxes (deep region) and 16-row boxes (window tiles at depth R); ring
-// planes (rows = L*Bmax*H*(R-1)*Wcap) in 16-row boxes.  Rows past the end of a
-// view read as zeros.
+// planes (rows = L*Bmax*H*(R-1)*Wcap) in 16-row boxes; ring and deep planes again
+// in 8-row boxes for the persistent kernel.  Rows past the end of a view read as
+// zeros.
 int make_tensor_maps(ripe_cache_s* c) {
     const EncodeFn encode = encode_fn();
     if (!encode) return -1;
-    static_assert(sizeof(TMaps) == sizeof(c->tmaps) + sizeof(CUtensorMap), "tensor map bundle");
+    static_assert(sizeof(c->tmaps) == 10 * sizeof(CUtensorMap), "tensor map bundle");
     const cuuint64_t deep_rows = (cuuint64_t)c->L * c->Bmax * c->H * c->Tmax;
     const cuuint64_t ring_rows = (cuuint64_t)c->L * c->Bmax * c->H * (c->R - 1) * c->Wcap;
     if (deep_rows >= (1ull << 31) || ring_rows >= (1ull << 31)) return -2;
@@ -1168,13 +1172,17 @@ int make_tensor_maps(ripe_cache_s* c) {
     };
     // With no ring planes (R = 1) the ring maps are never used; they alias the deep planes.
     const bool ring = ring_rows > 0;
-    const Spec spec[6] = {{c->kdeep, deep_rows, (cuuint32_t)kN},
-                          {c->vdeep, deep_rows, (cuuint32_t)kN},
-                          {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
-                          {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
-                          {c->kdeep, deep_rows, (cuuint32_t)kWinKeys},
-                          {c->vdeep, deep_rows, (cuuint32_t)kWinKeys}};
-    for (int i = 0; i < 6; ++i) {
+    const Spec spec[10] = {{c->kdeep, deep_rows, (cuuint32_t)kN},
+                           {c->vdeep, deep_rows, (cuuint32_t)kN},
+                           {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
+                           {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
+                           {c->kdeep, deep_rows, (cuuint32_t)kWinKeys},
+                           {c->vdeep, deep_rows, (cuuint32_t)kWinKeys},
+                           {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, 8u},
+                           {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, 8u},
+                           {c->kdeep, deep_rows, 8u},
+                           {c->vdeep, deep_rows, 8u}};
+    for (int i = 0; i < 10; ++i) {
         const cuuint64_t dims[2] = {(cuuint64_t)c->d, spec[i].rows};
         const cuuint32_t box[2] = {32, spec[i].box_rows};
         CUresult r = encode(reinterpret_cast<CUtensorMap*>(c->tmaps[i]), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,

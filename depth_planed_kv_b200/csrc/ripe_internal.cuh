@@ -25,11 +25,16 @@ struct ripe_cache_s {
     // Verify scratch (per-split partial results), grown on demand.
     void* work;
     size_t work_bytes;
-    // TMA descriptors (CUtensorMap), when the fused sm_100a kernel serves this cache
+    // TMA descriptors (CUtensorMap), when the sm_100a kernels serve this cache
     // (bf16, d in {64, 96, 128}): deep K, V planes in 64-row boxes (deep region),
-    // ring K, V planes and deep K, V planes in 16-row boxes (window tiles).
-    alignas(64) unsigned char tmaps[6][128];
+    // ring K, V planes and deep K, V planes in 16-row boxes (window tiles of the
+    // cluster kernel), and the same four in 8-row boxes (window chunks of the
+    // persistent kernel).
+    alignas(64) unsigned char tmaps[10][128];
     bool tc_ready;
+    // Test hook (ripe_debug_stall_next_verify): clock cycles of a wait that nothing
+    // ends, taken by the next persistent-kernel verify; 0 = off.
+    std::atomic<long long> probe_cycles{0};
 };
 
 // Store geometry, passed by value to kernels.
@@ -69,6 +74,7 @@ struct BranchArgs {
     const int32_t* seq_ids;      // implicit form: nseq sequence ids
     int nbranch, nrows, k;       // k: tokens per branch in the implicit form
     int max_ntok;                // tokens per branch the launch grid covers
+    int sliding;                 // per-query sliding window (implicit form, persistent kernel)
 };
 
 struct Branch {

@@ -1,0 +1,1115 @@
+// ripe_persist_sm100.cu -- the all-depths verify of one layer (k draft tokens of
+// each listed sequence at every loop depth 1..R) as one persistent sm_100a kernel.
+//
+// What is computed (RIPE abstract, sentence introducing RIPE): row (token j,
+// depth r) of sequence b attends to positions [0, A) at the deepest plane R, to
+// the window positions [A, T) at plane r, and to draft tokens 0..j at plane r,
+// with A = min(ws_b, T).  The deep region [0, A) is the same for all k*R rows of a
+// sequence, so it is one stacked-query contraction on the tensor cores; each
+// (depth, 8-token) slice of rows has its own window and block keys.
+//
+// Work items, spread over one wave of CTAs (one CTA per SM):
+//   deep item (sequence g, head h, chunk c): keys [c*chunk, (c+1)*chunk) of the
+//     deep region for all k*R rows (the last chunk runs to the region's end).  S = Q K^T (tcgen05.mma, fp32 in TMEM), online
+//     softmax on CUDA cores, O += P V (tcgen05.mma, P read from TMEM); K, V by TMA
+//     through ST shared-memory stages.  Warps 0-3 own TMEM lanes (one row each),
+//     warp 4 lane 0 issues TMA, warp 5 allocates TMEM and its lane 0 issues MMAs.
+//     The first `pd` CTAs take deep items pd apart.
+//   window unit (g, h, r, 8-token slice q): the window keys at plane r (ring
+//     slots, or deep-plane rows for r = R) and the slice's draft-block keys, in
+//     chunks of KC keys.  One warp runs a unit: it loads a chunk into its own
+//     shared-memory stage (8-row TMA boxes where eight window keys sit contiguously
+//     in memory, 16-byte cp.async for the rest and for block keys), then
+//     S^T = K Q^T and O^T = V^T P^T on warp-level MMA tiles (m16n8k16: keys and
+//     channels on the 16-row side, the <= 8 query rows on the 8-column side).
+//     Every CTA takes a contiguous range of units: n_lo per deep CTA, n_hi per
+//     other CTA (the host balances the bytes).  A CTA without deep items turns
+//     its deep warps and deep stages into more window warps.
+//
+// Merge without waiting: every item and unit that finishes leaves its partial
+// result (m in log2 units, l, unnormalised o) in scratch, then arrives on the
+// counter of each 8-row slice it covered.  A slice expects one arrival per deep
+// chunk that holds keys plus one from its window unit; the last arrival combines
+// the slice's partials -- M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L --
+// writes O and the LSE, and resets the counter to zero for the next call.  An
+// arrival that sees it will be last (the counter already holds every other
+// arrival) skips writing its own partial.  No CTA ever waits for another.
+#include <cuda.h>
+
+#include <cstring>
+
+#include "ripe_launch.h"
+#include "ripe_verify.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+constexpr int kN = 64;           // deep keys per tile
+constexpr int kDeepWarps = 6;    // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr int kWR = 8;           // rows per window unit (the N of an m16n8k16 tile)
+constexpr int kMaxItems = 32;    // deep items per CTA
+constexpr int kMaxUnitsPerGroup = kPersistSlices;
+
+// Tensor maps: deep K, V in 64-row boxes (deep region); ring K, V and deep K, V in
+// 8-row boxes (window chunks); Q of this call as [rows][H][d] in 128-row boxes of
+// one head.  All 32 columns wide with the 64-byte swizzle.
+struct PMaps {
+    CUtensorMap dk, dv, wk, wv, rk, rv, q;
+};
+
+struct DeepItem {
+    int g, h, c, seq, kb, ke, E, ntiles;
+};
+
+// Scalars of a launch beyond the common verify arguments.
+struct PArgs {
+    int32_t* cnt;      // [nseq][H][kPersistSlices] arrival counters of the 8-row slices (zero between calls)
+    int pd;            // CTAs that take deep items
+    int n_lo, n_hi;    // window units per deep CTA / per other CTA
+    int ndeep;         // G * H * nsplit deep items
+    int nunits;        // G * H * R * ceil(k / 8) window units
+    // Test hook: when nonzero, the softmax warps of every deep CTA first wait, this
+    // many clock cycles at most, on a barrier nothing signals, so that the bounded
+    // wait runs out (RIPE_DEVERR_TIMEOUT) and the abort path runs.
+    long long probe_cycles;
+    // Per-query sliding window (RIPE abstract, fifth sentence, read per query):
+    // draft token j at position T + j reads positions T+j-W+1 .. T+j at its own
+    // depth, older ones at plane R; 0 = the store's window for every row.
+    int sliding;
+};
+
+template <int D, int MT, int ST, int NWW, int KC>
+struct PLayout {
+    static constexpr int NCH = D / 32;
+    static constexpr bool QT = MT == 1;  // Q of the deep region in TMEM (one M tile) or shared memory
+    static constexpr int Q_BYTES = QT ? 0 : MT * NCH * 8192;
+    static constexpr int KV_STAGE = NCH * 4096;  // 64 keys x 64 B per column chunk
+    static constexpr int KCB = KC * 64;          // one column chunk of a window chunk
+    static constexpr int WSTAGE = 2 * NCH * KCB;  // K chunks, then V chunks
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
+    static constexpr int OFF_W = OFF_V + ST * KV_STAGE;
+    static constexpr int OFF_WEND = OFF_W + NWW * WSTAGE;
+    static constexpr int THREADS = 32 * (kDeepWarps + NWW);
+    static constexpr int NWARPS = THREADS / 32;
+    // A CTA without deep items: window stages over the whole stage region.
+    static constexpr int NW_FULL = (OFF_WEND / WSTAGE) < NWARPS ? (OFF_WEND / WSTAGE) : NWARPS;
+    static constexpr int OFF_OST = OFF_WEND;  // epilogue staging of the softmax warps
+    static constexpr int OST_BYTES = 4 * 8 * (32 * 4 + 16);
+    static constexpr int OFF_BAR = OFF_OST + OST_BYTES;
+    // q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain, epi_done, probe
+    static constexpr int NBAR = 1 + 3 * ST + 9;
+    static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;  // one per warp (window stage)
+    static constexpr int OFF_MISC = OFF_WBAR + NWARPS * 8;
+    static constexpr int OFF_ITEMS = OFF_MISC + 64;
+    static constexpr int OFF_FLAGS = OFF_ITEMS + kMaxItems * (int)sizeof(DeepItem);
+    static constexpr int BYTES = OFF_FLAGS + 2 * kMaxUnitsPerGroup;
+    static constexpr int SMEM = BYTES + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
+    static constexpr uint32_t O_COL(int mt) { return (uint32_t)(MT * 2 * kN + mt * 128); }
+    static constexpr uint32_t Q_COL = 2 * kN + 128;
+    static_assert(WSTAGE % 1024 == 0 && KV_STAGE % 1024 == 0 && Q_BYTES % 1024 == 0, "stage alignment");
+    static_assert(KC % 16 == 0 && KC <= 80, "window chunk");
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* err) {
+    const bool ok = sm100::mbar_wait(bar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Named barrier over the four softmax warps (ids 0 is __syncthreads).
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Context of sequence slot g of an all-depths call: its id, committed length T,
+// deep-region length A and the arrivals E each of its slices expects; ok is
+// false for an id outside the store (reported once).
+struct GroupCtx {
+    int seq, T, A, E;
+    bool ok;
+};
+
+__device__ __forceinline__ GroupCtx group_ctx(const VerifyArgs& a, int g, bool report) {
+    GroupCtx c;
+    c.seq = a.ba.seq_ids[g];
+    c.ok = c.seq >= 0 && c.seq < a.s.Bmax;
+    if (!c.ok) {
+        if (report) set_device_error(a.s.err, RIPE_DEVERR_SEQ_RANGE);
+        c.T = c.A = 0;
+        c.E = 1;
+        return c;
+    }
+    c.T = context_length(a.s.len, a.ctx, a.s.err, c.seq, report);
+    c.A = min(a.s.ws[c.seq], c.T);
+    c.E = deep_splits_used(c.A, a.chunk, a.nsplit) + 1;
+    return c;
+}
+
+// Visibility of a window unit's key kk to row (token) j under the sliding window:
+// keys [0, nw) are window positions A + kk at plane r, [nw, nw + nblk) draft
+// tokens at plane r, then ndw window positions at plane R, then draft tokens at
+// plane R.  sbase = T - W + 1 - A is row 0's first plane-r position, minus A.
+__device__ __forceinline__ bool slide_visible(int kk, int j, int nw, int nblk, int ndw, int nk, int sbase, int W) {
+    if (kk < nw) return kk >= sbase + j;
+    if (kk < nw + nblk) {
+        const int jj = kk - nw;
+        return jj <= j && jj >= j - W + 1;
+    }
+    if (kk < nw + nblk + ndw) return kk - nw - nblk < sbase + j;
+    if (kk < nk) return kk - nw - nblk - ndw < j - W + 1;
+    return false;
+}
+
+// Counter of the slice holding row (token j, depth r) of group g, head h.
+__device__ __forceinline__ int32_t* slice_counter(const VerifyArgs& a, const PArgs& p, int g, int j, int r, int h) {
+    const int QS = (a.ba.k + kWR - 1) / kWR;
+    return p.cnt + ((int64_t)g * a.s.H + h) * kPersistSlices + (r - 1) * QS + j / kWR;
+}
+
+template <int D, int MT, int ST, int NWW, int KC>
+__global__ void __launch_bounds__(PLayout<D, MT, ST, NWW, KC>::THREADS, 1)
+persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
+    using Lay = PLayout<D, MT, ST, NWW, KC>;
+    using namespace sm100;
+    constexpr int NCH = Lay::NCH;
+    constexpr uint32_t IDESC_QK = idesc_bf16(128, kN, 0);
+    constexpr uint32_t IDESC_PV = idesc_bf16(128, D, 1);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = sm + Lay::OFF_Q;
+    uint8_t* sK = sm + Lay::OFF_K;
+    uint8_t* sV = sm + Lay::OFF_V;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* v_full = bars + 1 + ST;
+    uint64_t* kv_empty = bars + 1 + 2 * ST;
+    uint64_t* s_full = bars + 1 + 3 * ST;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* pv_done = s_full + 4;
+    uint64_t* drain = s_full + 6;
+    uint64_t* epi_done = s_full + 7;
+    uint64_t* probe = s_full + 8;  // never signalled (test hook)
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(sm + Lay::OFF_WBAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 4);
+    int* n_items_s = reinterpret_cast<int*>(sm + Lay::OFF_MISC + 8);
+    // Snapshots of the abort flag for the softmax warps: written by thread 0 before
+    // a named barrier, read by all four after it, so that they decide alike even if
+    // another role sets the flag in between.
+    volatile int* stop_snap = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 12);
+    DeepItem* items = reinterpret_cast<DeepItem*>(sm + Lay::OFF_ITEMS);
+    uint8_t* known_last = sm + Lay::OFF_FLAGS;
+    uint8_t* is_last = known_last + kMaxUnitsPerGroup;
+
+    const StoreView& s = a.s;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int cta = blockIdx.x;
+    const bool deep_cta = cta < pa.pd;
+    const int R = s.R, H = s.H, k = a.ba.k;
+    const int QS = (k + kWR - 1) / kWR;  // 8-token slices per depth
+    const int kR = k * R;
+
+    if (threadIdx.x == 0) {
+        if (deep_cta) {
+            mbar_init(q_full, 128);
+            for (int i = 0; i < ST; ++i) {
+                mbar_init(k_full + i, 1);
+                mbar_init(v_full + i, 1);
+                mbar_init(kv_empty + i, 1);
+            }
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(s_full + i, 1);
+                mbar_init(p_full + i, 128);
+                mbar_init(pv_done + i, 1);
+            }
+            mbar_init(drain, 1);
+            mbar_init(epi_done, 4);
+            mbar_init(probe, 1);
+        }
+        // Window stages: 32 cp.async arrivals (one per lane) + lane 0's expect_tx.
+        for (int i = 0; i < Lay::NWARPS; ++i) mbar_init(wbar + i, 33);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (deep_cta && warp == 5) {
+        tmem_alloc(tmem_slot, Lay::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (lane == 0 && warp == 4) {
+        prefetch_tmap(&tm.dk);
+        prefetch_tmap(&tm.dv);
+        prefetch_tmap(&tm.wk);
+        prefetch_tmap(&tm.wv);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = deep_cta ? *tmem_slot : 0u;
+
+    // Inputs, metadata and scratch may belong to the previous kernel in the stream.
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    // ---- this CTA's deep items: item i = cta + pd * t, decoded as (g, h, c)
+    if (deep_cta && warp == 0) {
+        const int i = cta + pa.pd * lane;
+        DeepItem it{};
+        const bool have = lane < kMaxItems && i < pa.ndeep;
+        if (have) {
+            it.c = i % a.nsplit;
+            it.h = (i / a.nsplit) % H;
+            it.g = i / (a.nsplit * H);
+            const GroupCtx gc = group_ctx(a, it.g, it.h == 0 && it.c == 0);
+            it.seq = gc.seq;
+            it.E = gc.E;
+            // The last chunk takes every key past the others, so any deep length is
+            // covered whatever the length the host planned for.
+            it.kb = it.c * a.chunk;
+            it.ke = !gc.ok ? 0 : it.c == a.nsplit - 1 ? gc.A : min(gc.A, it.kb + a.chunk);
+            it.ntiles = it.ke > it.kb ? (it.ke - it.kb + kN - 1) / kN : 0;
+        }
+        // Compact the items that hold keys (empty chunks neither compute nor arrive).
+        const unsigned m = __ballot_sync(0xffffffffu, have && it.ntiles > 0);
+        if (have && it.ntiles > 0) items[__popc(m & ((1u << lane) - 1))] = it;
+        if (lane == 0) *n_items_s = __popc(m);
+    }
+    __syncthreads();
+    const int n_items = deep_cta ? *n_items_s : 0;
+
+    // ======================================================== deep pipeline
+    if (deep_cta && warp < kDeepWarps) {
+        if (warp == 4) {
+            // -------------------------------------------- TMA producer
+            if (lane == 0) {
+                int it = 0;
+                bool ok = true;
+                for (int n = 0; n < n_items && ok; ++n) {
+                    const DeepItem& di = items[n];
+                    const int row_base = ((a.layer * s.Bmax + di.seq) * H + di.h) * s.Tmax + di.kb;
+                    for (int i = 0; i < di.ntiles; ++i, ++it) {
+                        const int st = it % ST;
+                        if (it >= ST && !mbar_wait(kv_empty + st, ((it / ST) - 1) & 1, abort_flag, s.err)) {
+                            ok = false;
+                            break;
+                        }
+                        const int y = row_base + i * kN;
+                        mbar_expect_tx(k_full + st, Lay::KV_STAGE);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c)
+                            tma_load_2d(sK + st * Lay::KV_STAGE + c * 4096, &tm.dk, 32 * c, y, k_full + st);
+                        mbar_expect_tx(v_full + st, Lay::KV_STAGE);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c)
+                            tma_load_2d(sV + st * Lay::KV_STAGE + c * 4096, &tm.dv, 32 * c, y, v_full + st);
+                    }
+                }
+                if (*abort_flag) {
+                    // Let the copies already issued land before the shared memory goes away.
+                    volatile int no_abort = 0;
+                    for (int t = it > ST ? it - ST : 0; t < it; ++t) {
+                        mbar_wait(k_full + t % ST, (t / ST) & 1, &no_abort, s.err);
+                        mbar_wait(v_full + t % ST, (t / ST) & 1, &no_abort, s.err);
+                    }
+                }
+            }
+        } else if (warp == 5) {
+            // -------------------------------------------- MMA issuer
+            if (lane == 0 && n_items > 0) {
+                const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV);
+                // P V of global tile t (tile ti of its item): P from the S buffer t & 1.
+                auto issue_pv = [&](int t, int ti) -> bool {
+                    const int st = t % ST, pb = t & 1;
+                    if (!mbar_wait(p_full + pb, (t >> 1) & 1, abort_flag, s.err)) return false;
+                    if (!mbar_wait(v_full + st, (t / ST) & 1, abort_flag, s.err)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                        for (int ks = 0; ks < kN / 16; ++ks) {
+                            const uint64_t bd =
+                                smem_desc(v0 + st * Lay::KV_STAGE + ks * 1024, kN * 64, 512, kLayoutSwizzle64B);
+                            mma_bf16_ts(tmem + Lay::O_COL(mt), tmem + Lay::S_COL(mt, pb) + ks * 8, bd, IDESC_PV,
+                                        (ti > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(kv_empty + st);
+                    mma_commit(pv_done + pb);
+                    return true;
+                };
+                bool ok = true;
+                int it = 0;
+                for (int n = 0; n < n_items && ok; ++n) {
+                    const int ntiles = items[n].ntiles;
+                    // Q of this item is in place (the previous item's epilogue is done with O).
+                    if (!mbar_wait(q_full, n & 1, abort_flag, s.err)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int i = 0; i < ntiles; ++i, ++it) {
+                        const int st = it % ST, sb = it & 1;
+                        if (!mbar_wait(k_full + st, (it / ST) & 1, abort_flag, s.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks & 1) * 32;
+                                const uint64_t bd = smem_desc(k0 + st * Lay::KV_STAGE + (ks >> 1) * 4096 + off, 16,
+                                                              512, kLayoutSwizzle64B);
+                                if constexpr (Lay::QT) {
+                                    mma_bf16_ts(tmem + Lay::S_COL(mt, sb), tmem + Lay::Q_COL + ks * 8, bd, IDESC_QK,
+                                                ks > 0 ? 1u : 0u);
+                                } else {
+                                    const uint64_t ad = smem_desc(q0 + mt * NCH * 8192 + (ks >> 1) * 8192 + off, 16,
+                                                                  512, kLayoutSwizzle64B);
+                                    mma_bf16(tmem + Lay::S_COL(mt, sb), ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+                                }
+                            }
+                        }
+                        mma_commit(s_full + sb);
+                        if (i > 0 && !(ok = issue_pv(it - 1, i - 1))) break;
+                    }
+                    if (ok) ok = issue_pv(it - 1, ntiles - 1);
+                }
+                volatile int no_abort = 0;
+                mma_commit(drain);
+                mbar_wait(drain, 0, &no_abort, s.err);
+            }
+        } else {
+            // -------------------------------------------- softmax + epilogue (warps 0-3)
+            const int t = threadIdx.x;  // TMEM lane = M row within a tile
+            const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+            const float c2 = a.scale_log2;
+            float m[MT], l[MT];
+            bool ok = true;
+            int it = 0;
+            // A failed wait (timeout or abort) skips the remaining work, but every
+            // softmax warp still passes the epilogue's named barriers of this item;
+            // the abort flag, set before any of them, ends the loop for all alike.
+            for (int n = 0; n < n_items; ++n) {
+                const DeepItem di = items[n];
+                const int grow0 = di.g * kR;  // first row of the group
+                // ---- Q of this item (the previous item's MMAs are done: its epilogue waited for them)
+                if constexpr (Lay::QT) {
+                    const bool vq = t < kR;
+                    const uint4* src = reinterpret_cast<const uint4*>(a.Q + ((int64_t)(grow0 + (vq ? t : 0)) * H + di.h) * D * 2);
+#pragma unroll
+                    for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const uint4 x = vq ? __ldg(src + c0 / 4 + v) : make_uint4(0, 0, 0, 0);
+                            w[4 * v] = x.x;
+                            w[4 * v + 1] = x.y;
+                            w[4 * v + 2] = x.z;
+                            w[4 * v + 3] = x.w;
+                        }
+                        tmem_st16(lane_addr + Lay::Q_COL + c0, w);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(q_full);
+                } else {
+                    if (t == 0) {
+                        const bool go = n == 0 || mbar_wait(epi_done, (n - 1) & 1, abort_flag, s.err);
+                        if (go) {
+                            mbar_expect_tx(q_full, MT * NCH * 8192);
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int c = 0; c < NCH; ++c)
+                                    tma_load_3d(sQ + mt * NCH * 8192 + c * 8192, &tm.q, 32 * c, di.h,
+                                                grow0 + mt * 128, q_full);
+                        }
+                    } else {
+                        mbar_arrive(q_full);
+                    }
+                }
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    m[mt] = -INFINITY;
+                    l[mt] = 0.f;
+                }
+                if (pa.probe_cycles > 0 && n == 0) {
+                    const bool got = mbar_wait_slow(probe, 0, abort_flag, s.err, pa.probe_cycles);
+                    ok = __all_sync(0xffffffffu, got) && ok;
+                }
+                for (int i = 0; i < di.ntiles && ok; ++i, ++it) {
+                    const int sb = it & 1;
+                    if (!warp_wait(s_full + sb, (it >> 1) & 1, abort_flag, s.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nvalid = min(kN, di.ke - (di.kb + i * kN));
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        float sc[kN];
+                        tmem_ld32(lane_addr + Lay::S_COL(mt, sb), sc);
+                        tmem_ld32(lane_addr + Lay::S_COL(mt, sb) + 32, sc + 32);
+                        tmem_wait_ld();
+                        if (nvalid < kN) {
+#pragma unroll
+                            for (int c = 0; c < kN; ++c)
+                                if (c >= nvalid) sc[c] = -INFINITY;
+                        }
+                        float m4[4] = {sc[0], sc[1], sc[2], sc[3]};
+#pragma unroll
+                        for (int c = 4; c < kN; c += 4) {
+                            m4[0] = fmaxf(m4[0], sc[c]);
+                            m4[1] = fmaxf(m4[1], sc[c + 1]);
+                            m4[2] = fmaxf(m4[2], sc[c + 2]);
+                            m4[3] = fmaxf(m4[3], sc[c + 3]);
+                        }
+                        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c2;
+                        // The running max moves only when it grows by more than 2^8.
+                        float alpha = 1.f;
+                        const bool grow = mx > m[mt] + 8.f;
+                        if (grow) {
+                            const float mn = fmaxf(mx, m[mt]);
+                            alpha = ex2(m[mt] - mn);
+                            m[mt] = mn;
+                        }
+                        const float nm = -m[mt];
+                        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                        float pw[kN / 2];
+#pragma unroll
+                        for (int c = 0; c < kN / 2; ++c) {
+                            const float x0 = ex2(fmaf(sc[2 * c], c2, nm));
+                            const float x1 = ex2(fmaf(sc[2 * c + 1], c2, nm));
+                            s4[c & 3] += x0 + x1;
+                            pw[c] = __uint_as_float(pack_bf16(x0, x1));
+                        }
+                        tmem_st32(lane_addr + Lay::S_COL(mt, sb), pw);
+                        l[mt] = l[mt] * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                        if (i > 0 && __any_sync(0xffffffffu, grow)) {
+                            if (!warp_wait(pv_done + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, s.err)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int c0 = 0; c0 < D; c0 += 32) {
+                                float o[32];
+                                tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int c = 0; c < 32; ++c) o[c] *= alpha;
+                                tmem_st32(lane_addr + Lay::O_COL(mt) + c0, o);
+                            }
+                            tmem_wait_st();
+                        }
+                    }
+                    if (!ok) break;
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(p_full + sb);
+                }
+                // ---- epilogue of the item.  Slices that already hold every other
+                // arrival are merged here without writing this chunk's partial.
+                const int nslices = R * QS;
+                for (int u = t; u < nslices; u += 128) {
+                    const int r = u / QS + 1, q = u % QS;
+                    known_last[u] = ld_acquire(slice_counter(a, pa, di.g, q * kWR, r, di.h)) == di.E - 1;
+                }
+                if (ok) ok = warp_wait(pv_done + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, s.err);
+                tc_fence_after();
+                softmax_bar();
+                // Row (token j, depth r) of M row t in tile mt; its slice index.
+                int rows[MT], sl[MT];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int rl = mt * 128 + t;
+                    rows[mt] = rl < kR ? grow0 + rl : -1;
+                    sl[mt] = rl < kR ? ((rl % R) * QS + (rl / R) / kWR) : 0;
+                }
+                // Publish the partial of every row whose slice is not known to end here:
+                // 8 rows x 32 columns at a time staged in shared memory, 128-byte pieces.
+                {
+                    constexpr int OSTR = 32 * 4 + 16;
+                    uint8_t* ostage = sm + Lay::OFF_OST + warp * 8 * OSTR;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const bool pub = ok && rows[mt] >= 0 && !known_last[sl[mt]];
+                        const int64_t pi = pub ? ((int64_t)rows[mt] * H + di.h) * a.nseg + di.c : -1;
+                        if (pub) a.part_ml[pi] = make_float2(m[mt], l[mt]);
+                        if (!__any_sync(0xffffffffu, pub)) continue;
+#pragma unroll 1
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            float o[32];
+                            tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int part = 0; part < 4; ++part) {
+                                if ((lane >> 3) == part) {
+                                    float4* d4 = reinterpret_cast<float4*>(ostage + (lane & 7) * OSTR);
+#pragma unroll
+                                    for (int c = 0; c < 8; ++c)
+                                        d4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                                }
+                                __syncwarp();
+#pragma unroll
+                                for (int e0 = 0; e0 < 8 * 8; e0 += 32) {
+                                    const int e = e0 + lane, kr = e >> 3, c4 = e & 7;
+                                    const int64_t pk = __shfl_sync(0xffffffffu, pi, part * 8 + kr);
+                                    if (pk >= 0)
+                                        reinterpret_cast<float4*>(a.part_o + pk * D + c0)[c4] =
+                                            *reinterpret_cast<const float4*>(ostage + kr * OSTR + c4 * 16);
+                                }
+                                __syncwarp();
+                            }
+                        }
+                    }
+                }
+                __threadfence();
+                if (t == 0) *stop_snap = *abort_flag;
+                softmax_bar();
+                const bool all_ok = !*stop_snap;
+                for (int u = t; u < nslices; u += 128) {
+                    const int r = u / QS + 1, q = u % QS;
+                    int32_t* cp = slice_counter(a, pa, di.g, q * kWR, r, di.h);
+                    bool last = false;
+                    if (all_ok) {
+                        last = known_last[u];
+                        if (!last) last = atomicAdd(cp, 1) == di.E - 1;
+                        if (last) *cp = 0;  // the last arrival: nothing else touches it in this call
+                    }
+                    is_last[u] = last;
+                }
+                __threadfence();
+                softmax_bar();
+                // Merge the rows of the slices that ended here: this chunk's partial from
+                // TMEM and registers, the other deep chunks' and the window's from scratch.
+                // Segments in the fixed order (deep chunks, then the window) whoever
+                // merges, so the result does not depend on which arrival came last.
+                // tcgen05.ld is warp-collective: a warp loads O when any of its rows
+                // merges, and only those rows use it.
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const bool mine = rows[mt] >= 0 && is_last[sl[mt]];
+                    if (!__any_sync(0xffffffffu, mine)) continue;
+                    const int64_t ro = mine ? (int64_t)rows[mt] * H + di.h : 0;
+                    const int np = mine ? di.E - 1 : 0;  // deep chunks with keys; segment np is the window
+                    float2 ml[9];
+                    float M = -INFINITY;
+                    for (int sg = 0; sg <= np; ++sg) {
+                        ml[sg] = sg == di.c ? make_float2(m[mt], l[mt])
+                                            : __ldcg(a.part_ml + ro * a.nseg + (sg < np ? sg : a.nsplit));
+                        M = fmaxf(M, ml[sg].x);
+                    }
+                    float fs[9], L = 0.f;
+                    for (int sg = 0; sg <= np; ++sg) {
+                        fs[sg] = ex2(ml[sg].x - M);
+                        L = fmaf(ml[sg].y, fs[sg], L);
+                    }
+                    const float inv = 1.f / L;
+                    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        float own[32], acc[32];
+                        tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, own);
+                        tmem_wait_ld();
+                        if (!mine) continue;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+                        for (int sg = 0; sg <= np; ++sg) {
+                            const float f = fs[sg];
+                            if (sg == di.c) {
+#pragma unroll
+                                for (int c = 0; c < 32; ++c) acc[c] = fmaf(own[c], f, acc[c]);
+                                continue;
+                            }
+                            const float4* src = reinterpret_cast<const float4*>(
+                                a.part_o + (ro * a.nseg + (sg < np ? sg : a.nsplit)) * D + c0);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const float4 x = __ldcg(src + c);
+                                acc[4 * c] = fmaf(x.x, f, acc[4 * c]);
+                                acc[4 * c + 1] = fmaf(x.y, f, acc[4 * c + 1]);
+                                acc[4 * c + 2] = fmaf(x.z, f, acc[4 * c + 2]);
+                                acc[4 * c + 3] = fmaf(x.w, f, acc[4 * c + 3]);
+                            }
+                        }
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            reinterpret_cast<uint4*>(orow + c0)[c] =
+                                make_uint4(pack_bf16(acc[8 * c] * inv, acc[8 * c + 1] * inv),
+                                           pack_bf16(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
+                                           pack_bf16(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
+                                           pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+                    }
+                    if (mine && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
+                }
+                tc_fence_before();
+                __syncwarp();
+                // The epilogue is done with O and (MT = 2) with the Q buffer's staging.
+                fence_proxy_async_smem();
+                if (lane == 0) mbar_arrive(epi_done);
+                if (t == 0) *stop_snap = *abort_flag;
+                softmax_bar();  // the flags are rewritten by the next item
+                if (*stop_snap) break;
+            }
+        }
+    }
+
+    // ======================================================== window units
+    // Deep CTA: warps 6.. with stages after the deep ones.  Other CTAs: every warp
+    // with a stage anywhere in the stage region.
+    const int wbase = deep_cta ? kDeepWarps : 0;
+    const int nww = deep_cta ? NWW : Lay::NW_FULL;
+    const int wi = warp - wbase;
+    if (wi >= 0 && wi < nww) {
+        uint8_t* stage = sm + (deep_cta ? Lay::OFF_W + wi * Lay::WSTAGE : wi * Lay::WSTAGE);
+        uint64_t* bar = wbar + warp;
+        const uint32_t stage_a = smem_u32(stage);
+        const int64_t ub64 = cta < pa.pd ? (int64_t)cta * pa.n_lo
+                                         : (int64_t)pa.pd * pa.n_lo + (int64_t)(cta - pa.pd) * pa.n_hi;
+        const int64_t ue64 = ub64 + (cta < pa.pd ? pa.n_lo : pa.n_hi);
+        const int ubeg = (int)(ub64 < pa.nunits ? ub64 : pa.nunits);
+        const int uend = (int)(ue64 < pa.nunits ? ue64 : pa.nunits);
+        constexpr int NKS = D / 16, NMT = D / 16, NT = KC / 16;
+        const float c2 = a.scale_log2;
+        const int q4 = lane & 3, r8 = lane >> 2;
+        const int ra = 2 * q4, rb = ra + 1;
+        // ldmatrix row addresses in the swizzled layout (K: A operand, rows = keys;
+        // V: A operand of O^T by .trans).
+        const int rk = (lane & 7) + 8 * ((lane >> 3) & 1), rv = (lane & 7) + 8 * (lane >> 4);
+        const uint32_t k_sw0 = (((lane >> 4) + 0) ^ ((rk >> 1) & 3)) << 4;
+        const uint32_t k_sw1 = (((lane >> 4) + 2) ^ ((rk >> 1) & 3)) << 4;
+        const uint32_t v_sw0 = ((((lane >> 3) & 1) + 0) ^ ((rv >> 1) & 3)) << 4;
+        const uint32_t v_sw1 = ((((lane >> 3) & 1) + 2) ^ ((rv >> 1) & 3)) << 4;
+        int cached_g = -1;
+        GroupCtx gc{};
+        uint32_t phase = 0;
+        bool wok = true;
+        for (int u = ubeg + wi; u < uend && wok; u += nww) {
+            const int q = u % QS;
+            const int r = (u / QS) % R + 1;
+            const int h = (u / (QS * R)) % H;
+            const int g = u / (QS * R * H);
+            if (g != cached_g) {
+                gc = group_ctx(a, g, false);
+                cached_g = g;
+            }
+            if (!gc.ok) continue;
+            const int j0 = q * kWR, nr = min(kWR, k - j0);
+            const int nw = gc.T - gc.A, nblk = j0 + nr;
+            const bool ring = r < R;
+            // Sliding window (depth r < R only; at depth R both readings agree): row j
+            // reads window position p at plane r iff p >= T + j - W + 1, else at plane
+            // R, and draft token j' at plane r iff j' >= j - W + 1, else its depth-R
+            // row.  The unit's keys then continue with plane-R copies of the first
+            // window positions (ndw) and the depth-R rows of the first draft tokens
+            // (nbr), each masked per row.
+            const bool slide = pa.sliding && ring;
+            const int sbase = gc.T - s.W + 1 - gc.A;  // (T + j - W + 1) - A at j = 0
+            const int ndw = slide ? max(0, min(nw, sbase + j0 + nr - 1)) : 0;
+            const int nbr = slide ? max(0, j0 + nr - s.W) : 0;
+            const int nk = nw + nblk + ndw + nbr;
+            const int slot0 = gc.A % s.Wcap;
+            const int64_t grow0 = (int64_t)g * kR;
+            // Q^T fragments (B operand): Q[j0 + lane/4][16 ks + 2 q4 ..] and 8 channels on.
+            uint32_t bq[NKS][2];
+            {
+                const bool okq = r8 < nr;
+                const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+                    a.Q + (okq ? ((grow0 + (int64_t)(j0 + r8) * R + r - 1) * H + h) * (2 * D) : 0));
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    bq[ks][0] = okq ? __ldg(qp + 8 * ks + q4) : 0u;
+                    bq[ks][1] = okq ? __ldg(qp + 8 * ks + 4 + q4) : 0u;
+                }
+            }
+            float o[NMT][4];
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+            float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+            // Global rows of the ring plane r (slot 0) / of the deep plane (position 0),
+            // in the tensor maps' 2-D views, and byte bases for the per-key copies.
+            const int64_t ring_y = ((((int64_t)a.layer * s.Bmax + gc.seq) * H + h) * (R - 1) + (r - 1)) * s.Wcap;
+            const int64_t deep_y = (((int64_t)a.layer * s.Bmax + gc.seq) * H + h) * s.Tmax;
+            for (int k0 = 0; k0 < nk; k0 += KC) {
+                const int kc = min(KC, nk - k0);
+                const int nt = (kc + 15) / 16;
+                // ---- load keys [k0, k0 + 16 nt) into the stage: 8-key groups of window
+                // keys contiguous in memory by TMA, the rest (a wrapping group, a
+                // partial group, block keys, zero fill) by 16-byte copies.
+                __syncwarp();
+                fence_proxy_async_smem();  // earlier reads of this stage come before new writes
+                uint32_t tma_groups = 0;   // bit m: group m of this chunk goes by TMA
+#pragma unroll
+                for (int gm = 0; gm < 2 * NT; ++gm) {
+                    const int kk = k0 + 8 * gm;
+                    if (gm < 2 * nt && kk + 8 <= nw) {
+                        const bool contig = !ring || ((slot0 + kk) % s.Wcap) + 8 <= s.Wcap;
+                        if (contig) tma_groups |= 1u << gm;
+                    }
+                }
+                if (lane == 0) {
+                    mbar_expect_tx(bar, (uint32_t)__popc(tma_groups) * 8 * 64 * NCH * 2);
+                    uint32_t gmask = tma_groups;
+                    while (gmask) {
+                        const int gm = __ffs(gmask) - 1;
+                        gmask &= gmask - 1;
+                        const int kk = k0 + 8 * gm;
+                        const int y = ring ? (int)(ring_y + (slot0 + kk) % s.Wcap) : (int)(deep_y + gc.A + kk);
+                        const CUtensorMap* mk = ring ? &tm.wk : &tm.rk;
+                        const CUtensorMap* mv = ring ? &tm.wv : &tm.rv;
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c) {
+                            tma_load_2d(stage + c * Lay::KCB + gm * 512, mk, 32 * c, y, bar);
+                            tma_load_2d(stage + (NCH + c) * Lay::KCB + gm * 512, mv, 32 * c, y, bar);
+                        }
+                    }
+                }
+                // Per-key copies: (key, 16-byte vector) pairs of the other groups.
+                {
+                    constexpr int VPR = NCH * 4;  // 16-byte vectors per key row
+                    const uint32_t other = ((1u << (2 * nt)) - 1) & ~tma_groups;
+                    const int nother = __popc(other);
+                    for (int e = lane; e < nother * 8 * VPR; e += 32) {
+                        const int gi = e / (8 * VPR), rem = e % (8 * VPR);
+                        const int kr = rem / VPR, v = rem % VPR;
+                        // gi-th set bit of `other`
+                        uint32_t om = other;
+                        for (int z = 0; z < gi; ++z) om &= om - 1;
+                        const int gm = __ffs(om) - 1;
+                        const int kl = 8 * gm + kr;  // key within the chunk
+                        const int kk = k0 + kl;
+                        const char* ks_ = a.Q;
+                        const char* vs_ = a.Q;
+                        bool valid = true;
+                        if (kk < nw) {
+                            const int64_t row = ring ? ring_y + (slot0 + kk) % s.Wcap : deep_y + gc.A + kk;
+                            const int64_t off = row * (2 * D) + v * 16;
+                            ks_ = (ring ? s.kwin : s.kdeep) + off;
+                            vs_ = (ring ? s.vwin : s.vdeep) + off;
+                        } else if (kk < nw + nblk) {
+                            const int64_t off = ((grow0 + (int64_t)(kk - nw) * R + r - 1) * H + h) * (2 * D) + v * 16;
+                            ks_ = a.Kb + off;
+                            vs_ = a.Vb + off;
+                        } else if (kk < nw + nblk + ndw) {  // sliding: window position at plane R
+                            const int64_t off = (deep_y + gc.A + (kk - nw - nblk)) * (2 * D) + v * 16;
+                            ks_ = s.kdeep + off;
+                            vs_ = s.vdeep + off;
+                        } else if (kk < nk) {  // sliding: draft token at plane R (its depth-R row)
+                            const int64_t off =
+                                ((grow0 + (int64_t)(kk - nw - nblk - ndw) * R + R - 1) * H + h) * (2 * D) + v * 16;
+                            ks_ = a.Kb + off;
+                            vs_ = a.Vb + off;
+                        } else {
+                            valid = false;
+                        }
+                        const int c = v >> 2, v4 = v & 3;
+                        uint8_t* dk = stage + c * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4);
+                        cp_async16_zfill(dk, ks_, valid);
+                        cp_async16_zfill(dk + NCH * Lay::KCB, vs_, valid);
+                    }
+                    cp_async_mbar_arrive(bar);
+                }
+                if (!warp_wait(bar, phase & 1, abort_flag, s.err)) {
+                    wok = false;
+                    break;
+                }
+                ++phase;
+                const uint32_t sb = smem_ready(stage_a);
+                // ---- S^T = K Q^T for the chunk's 16-key tiles (independent chains)
+                float sc[NT][4];
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt) {
+                    sc[tt][0] = sc[tt][1] = sc[tt][2] = sc[tt][3] = 0.f;
+                    if (tt < nt) {
+#pragma unroll
+                        for (int ks = 0; ks < NKS; ++ks) {
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4_r(sb + (ks >> 1) * Lay::KCB + (16 * tt + rk) * 64 + ((ks & 1) ? k_sw1 : k_sw0), a0,
+                                      a1, a2, a3);
+                            mma_16816(sc[tt], a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+                        }
+                    }
+                }
+                // ---- visibility and the chunk's row maxima.  Key kk is visible to row j
+                // if it is a window key, or block token kk - nw <= j.
+                float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt) {
+                    if (tt < nt) {
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int kk = k0 + 16 * tt + r8 + 8 * hf;
+                            bool va, vb;
+                            if (!slide) {
+                                va = kk < nw || (kk < nk && kk - nw <= j0 + ra);
+                                vb = kk < nw || (kk < nk && kk - nw <= j0 + rb);
+                            } else {
+                                va = slide_visible(kk, j0 + ra, nw, nblk, ndw, nk, sbase, s.W);
+                                vb = slide_visible(kk, j0 + rb, nw, nblk, ndw, nk, sbase, s.W);
+                            }
+                            float& xa = sc[tt][2 * hf];
+                            float& xb = sc[tt][2 * hf + 1];
+                            xa = va ? xa * c2 : -INFINITY;
+                            xb = vb ? xb * c2 : -INFINITY;
+                            mx_a = fmaxf(mx_a, xa);
+                            mx_b = fmaxf(mx_b, xb);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, o2));
+                    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, o2));
+                }
+                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+                const float al_a = mn_a == -INFINITY ? 1.f : ex2(m_a - mn_a);
+                const float al_b = mn_b == -INFINITY ? 1.f : ex2(m_b - mn_b);
+                m_a = mn_a;
+                m_b = mn_b;
+                l_a *= al_a;
+                l_b *= al_b;
+#pragma unroll
+                for (int mt = 0; mt < NMT; ++mt) {
+                    o[mt][0] *= al_a;
+                    o[mt][2] *= al_a;
+                    o[mt][1] *= al_b;
+                    o[mt][3] *= al_b;
+                }
+                // ---- probabilities and P^T fragments (8x8 transposes of the S^T fragments)
+                uint32_t pb[NT][2];
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt) {
+                    if (tt < nt) {
+                        const float p0 = mn_a == -INFINITY ? 0.f : ex2(sc[tt][0] - mn_a);
+                        const float p1 = mn_b == -INFINITY ? 0.f : ex2(sc[tt][1] - mn_b);
+                        const float p2 = mn_a == -INFINITY ? 0.f : ex2(sc[tt][2] - mn_a);
+                        const float p3 = mn_b == -INFINITY ? 0.f : ex2(sc[tt][3] - mn_b);
+                        l_a += p0 + p2;
+                        l_b += p1 + p3;
+                        pb[tt][0] = movmatrix_t(pack_bf16(p0, p1));
+                        pb[tt][1] = movmatrix_t(pack_bf16(p2, p3));
+                    } else {
+                        pb[tt][0] = pb[tt][1] = 0u;
+                    }
+                }
+                // ---- O^T += V^T P^T (one chain per 16-channel tile)
+#pragma unroll
+                for (int mt = 0; mt < NMT; ++mt) {
+#pragma unroll
+                    for (int tt = 0; tt < NT; ++tt) {
+                        if (tt < nt) {
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4_t_r(sb + NCH * Lay::KCB + (mt >> 1) * Lay::KCB + (16 * tt + rv) * 64 +
+                                            ((mt & 1) ? v_sw1 : v_sw0),
+                                        a0, a1, a2, a3);
+                            mma_16816(o[mt], a0, a1, a2, a3, pb[tt][0], pb[tt][1]);
+                        }
+                    }
+                }
+            }
+            if (!wok) break;
+            // ---- the unit's end: row sums across the lanes of a row
+#pragma unroll
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                l_a += __shfl_xor_sync(0xffffffffu, l_a, o2);
+                l_b += __shfl_xor_sync(0xffffffffu, l_b, o2);
+            }
+            int32_t* cp = slice_counter(a, pa, g, j0, r, h);
+            bool last = false;
+            if (lane == 0) last = ld_acquire(cp) == gc.E - 1;
+            last = __shfl_sync(0xffffffffu, last, 0);
+            const bool va = ra < nr, vb = rb < nr;
+            const int64_t ro_a = (grow0 + (int64_t)(j0 + ra) * R + r - 1) * H + h;
+            const int64_t ro_b = (grow0 + (int64_t)(j0 + rb) * R + r - 1) * H + h;
+            if (!last) {
+                // Publish this unit's partial (segment nsplit), then arrive.
+                const int64_t pa_ = ro_a * a.nseg + a.nsplit, pb_ = ro_b * a.nseg + a.nsplit;
+#pragma unroll
+                for (int mt = 0; mt < NMT; ++mt) {
+                    const int ch = 16 * mt + r8;
+                    if (va) {
+                        a.part_o[pa_ * D + ch] = o[mt][0];
+                        a.part_o[pa_ * D + ch + 8] = o[mt][2];
+                    }
+                    if (vb) {
+                        a.part_o[pb_ * D + ch] = o[mt][1];
+                        a.part_o[pb_ * D + ch + 8] = o[mt][3];
+                    }
+                }
+                if (r8 == 0) {
+                    if (va) a.part_ml[pa_] = make_float2(m_a, l_a);
+                    if (vb) a.part_ml[pb_] = make_float2(m_b, l_b);
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) last = atomicAdd(cp, 1) == gc.E - 1;
+                last = __shfl_sync(0xffffffffu, last, 0);
+            }
+            if (!last) continue;
+            if (lane == 0) *cp = 0;
+            __threadfence();
+            // ---- merge rows ra, rb of this lane's channels with the deep chunks'
+            // partials, segments in the fixed order (deep chunks, then this window).
+            const int np = gc.E - 1;
+            float Ma = m_a, Mb = m_b;
+            for (int sg = 0; sg < np; ++sg) {
+                if (va) Ma = fmaxf(Ma, __ldcg(a.part_ml + ro_a * a.nseg + sg).x);
+                if (vb) Mb = fmaxf(Mb, __ldcg(a.part_ml + ro_b * a.nseg + sg).x);
+            }
+            float acc[NMT][4];
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+            float La = 0.f, Lb = 0.f;
+            for (int sg = 0; sg < np; ++sg) {
+                if (va) {
+                    const float2 ml = __ldcg(a.part_ml + ro_a * a.nseg + sg);
+                    const float f = ex2(ml.x - Ma);
+                    La = fmaf(ml.y, f, La);
+                    const float* po = a.part_o + (ro_a * a.nseg + sg) * D + r8;
+#pragma unroll
+                    for (int mt = 0; mt < NMT; ++mt) {
+                        acc[mt][0] = fmaf(__ldcg(po + 16 * mt), f, acc[mt][0]);
+                        acc[mt][2] = fmaf(__ldcg(po + 16 * mt + 8), f, acc[mt][2]);
+                    }
+                }
+                if (vb) {
+                    const float2 ml = __ldcg(a.part_ml + ro_b * a.nseg + sg);
+                    const float f = ex2(ml.x - Mb);
+                    Lb = fmaf(ml.y, f, Lb);
+                    const float* po = a.part_o + (ro_b * a.nseg + sg) * D + r8;
+#pragma unroll
+                    for (int mt = 0; mt < NMT; ++mt) {
+                        acc[mt][1] = fmaf(__ldcg(po + 16 * mt), f, acc[mt][1]);
+                        acc[mt][3] = fmaf(__ldcg(po + 16 * mt + 8), f, acc[mt][3]);
+                    }
+                }
+            }
+            const float fa = ex2(m_a - Ma), fb = ex2(m_b - Mb);
+            La = fmaf(l_a, fa, La);
+            Lb = fmaf(l_b, fb, Lb);
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt) {
+                o[mt][0] = fmaf(o[mt][0], fa, acc[mt][0]);
+                o[mt][2] = fmaf(o[mt][2], fa, acc[mt][2]);
+                o[mt][1] = fmaf(o[mt][1], fb, acc[mt][1]);
+                o[mt][3] = fmaf(o[mt][3], fb, acc[mt][3]);
+            }
+            const float ia = 1.f / La, ib = 1.f / Lb;
+            __nv_bfloat16* Oa = reinterpret_cast<__nv_bfloat16*>(a.O) + ro_a * D + r8;
+            __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(a.O) + ro_b * D + r8;
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt) {
+                if (va) {
+                    Oa[16 * mt] = __float2bfloat16_rn(o[mt][0] * ia);
+                    Oa[16 * mt + 8] = __float2bfloat16_rn(o[mt][2] * ia);
+                }
+                if (vb) {
+                    Ob[16 * mt] = __float2bfloat16_rn(o[mt][1] * ib);
+                    Ob[16 * mt + 8] = __float2bfloat16_rn(o[mt][3] * ib);
+                }
+            }
+            if (r8 == 0 && a.lse) {
+                if (va) a.lse[ro_a] = (Ma + log2f(La)) * 0.69314718055994531f;
+                if (vb) a.lse[ro_b] = (Mb + log2f(Lb)) * 0.69314718055994531f;
+            }
+        }
+        if (!wok) {
+            // Let this warp's copies land before the CTA's shared memory goes away.
+            volatile int no_abort = 0;
+            cp_async_wait_all();
+            mbar_wait(bar, phase & 1, &no_abort, s.err);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (deep_cta && warp == 5) tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+template <int D, int MT, int ST, int NWW, int KC>
+cudaError_t launch_p(const PMaps& tm, const VerifyArgs& a, const PArgs& pa, int grid, cudaStream_t st) {
+    using Lay = PLayout<D, MT, ST, NWW, KC>;
+    static_assert(Lay::SMEM <= 232448, "shared memory budget");
+    static PerDeviceOnce configured;
+    cudaError_t ce = per_device_once(configured, [] {
+        cudaError_t e = cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+        if (e != cudaSuccess) return e;
+        return cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC>,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    });
+    if (ce != cudaSuccess) return ce;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(Lay::THREADS);
+    cfg.dynamicSmemBytes = Lay::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, persist_kernel<D, MT, ST, NWW, KC>, tm, a, pa);
+    ripe_count_launch();
+    return e;
+}
+
+}  // namespace
+
+// Window warps a CTA of each role runs, for the planner's cost model.
+void persist_shape(int d, int mt, int* nww_deep, int* nww_other) {
+#define RIPE_SHAPE(D_, MT_, ST_, NWW_, KC_)                      \
+    if (d == D_ && mt == MT_) {                                  \
+        *nww_deep = NWW_;                                        \
+        *nww_other = PLayout<D_, MT_, ST_, NWW_, KC_>::NW_FULL;  \
+        return;                                                  \
+    }
+    RIPE_SHAPE(64, 1, 4, 6, 80)
+    RIPE_SHAPE(96, 1, 4, 4, 80)
+    RIPE_SHAPE(128, 1, 3, 3, 80)
+    RIPE_SHAPE(64, 2, 4, 5, 80)
+    RIPE_SHAPE(96, 2, 3, 3, 80)
+    RIPE_SHAPE(128, 2, 3, 2, 48)
+#undef RIPE_SHAPE
+    *nww_deep = *nww_other = 0;
+}
+
+cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int32_t* cnt, int pd, int n_lo, int n_hi,
+                           int ndeep, int nunits, int grid, int mt, long long probe_cycles, int sliding,
+                           cudaStream_t st) {
+    // Cache maps: 0 deep K, 1 deep V (64-row boxes); 6 ring K, 7 ring V, 8 deep K,
+    // 9 deep V (8-row boxes); plus one of this call's Q.
+    PMaps tm;
+    const CUtensorMap* cm = reinterpret_cast<const CUtensorMap*>(tmaps);
+    tm.dk = cm[0];
+    tm.dv = cm[1];
+    tm.wk = cm[6];
+    tm.wv = cm[7];
+    tm.rk = cm[8];
+    tm.rv = cm[9];
+    VerifyArgs a = args;
+    if (!make_q_map(&tm.q, a)) return cudaErrorInvalidValue;
+    PArgs pa{cnt, pd, n_lo, n_hi, ndeep, nunits, probe_cycles, sliding};
+    const int d = a.s.d;
+    if (mt == 1) {
+        if (d == 64) return launch_p<64, 1, 4, 6, 80>(tm, a, pa, grid, st);
+        if (d == 96) return launch_p<96, 1, 4, 4, 80>(tm, a, pa, grid, st);
+        if (d == 128) return launch_p<128, 1, 3, 3, 80>(tm, a, pa, grid, st);
+    } else {
+        if (d == 64) return launch_p<64, 2, 4, 5, 80>(tm, a, pa, grid, st);
+        if (d == 96) return launch_p<96, 2, 3, 3, 80>(tm, a, pa, grid, st);
+        if (d == 128) return launch_p<128, 2, 3, 2, 48>(tm, a, pa, grid, st);
+    }
+    return cudaErrorInvalidValue;
+}

@@ -389,7 +389,102 @@ cudaError_t launch_seg(const VerifyArgs& a, int seg_first, int seg_count, int nb
     return cudaGetLastError();
 }
 
+// The persistent kernel serves an all-depths call whose k*R rows of a sequence
+// fit two 128-row M tiles and whose (depth, 8-token) slices fit the counter
+// layout.  The plan splits the deep region into nsplit chunks and balances the
+// bytes each CTA streams: pd CTAs take deep items (sequence, head, chunk) pd
+// apart plus n_lo window units each; the others take n_hi window units.  A deep
+// item also costs a fixed latency (Q load, pipeline fill, epilogue), counted as
+// bytes of streaming.  The kernel's last chunk runs to the end of the deep
+// region, so the chunk length only shapes the balance: it is sized for the
+// deep region an evicted store has at the host's length bound (len_ub - W).
+bool plan_persist(const ripe_cache_s* c, int nseq, int k, int len_ub, VerifyPlan& p) {
+    const int A_ub = len_ub - c->W > 0 ? len_ub - c->W : 0;
+    const int R = c->R, H = c->H, d = c->d;
+    const int kR = k * R, QS = (k + 7) / 8;
+    if (kR > 256 || R * QS > kPersistSlices || nseq < 1) return false;
+    const int mt = kR > 128 ? 2 : 1;
+    int nww_deep = 0, nww_other = 0;
+    persist_shape(d, mt, &nww_deep, &nww_other);
+    if (nww_other == 0) return false;
+    const int P = device_sm_count();
+    if (P < 1) return false;
+    const double kv = 4.0 * d, row = 2.0 * d;
+    const int wl = len_ub < c->W ? len_ub : c->W;
+    const double bU = (wl + k) * kv + 2.0 * (k < 8 ? k : 8) * row;
+    const double item_fixed = 96e3;
+    const int64_t NU = (int64_t)nseq * H * R * QS;
+    if (NU > (1 << 30)) return false;
+    double best = 1e300;
+    bool found = false;
+    for (int nd = 1; nd <= 8; ++nd) {
+        int chunk = (A_ub + nd - 1) / nd;
+        chunk = (chunk + 63) / 64 * 64;
+        if (chunk < 64) chunk = 64;
+        if (nd > 1 && (int64_t)chunk * (nd - 1) >= A_ub) break;  // a chunk would always be empty
+        const int64_t ND = (int64_t)nseq * H * nd;
+        const int pd = (int)(ND < P ? ND : P);
+        const int64_t I = (ND + pd - 1) / pd;
+        if (I > 32) continue;
+        const double bD = chunk * kv + kR * row + item_fixed;
+        const double LD = I * bD;
+        int64_t n_lo, n_hi;
+        double Tm;
+        if (pd == P) {
+            n_hi = 0;
+            n_lo = (NU + P - 1) / P;
+            Tm = LD + n_lo * bU;
+        } else {
+            const double T0 = LD > (ND * bD + NU * bU) / P ? LD : (ND * bD + NU * bU) / P;
+            n_hi = (int64_t)ceil(T0 / bU);
+            if (n_hi < 1) n_hi = 1;
+            for (;;) {
+                const double spare = n_hi * bU - LD;
+                n_lo = spare > 0 ? (int64_t)floor(spare / bU) : 0;
+                if (pd * n_lo + (int64_t)(P - pd) * n_hi >= NU) break;
+                ++n_hi;
+            }
+            Tm = LD + n_lo * bU > n_hi * bU ? LD + n_lo * bU : n_hi * bU;
+        }
+        if (Tm < 0.98 * best) {  // more chunks only for a clear gain (their partials cost traffic)
+            best = Tm;
+            found = true;
+            p.nsplit = nd;
+            p.chunk = chunk;
+            p.pd = pd;
+            p.n_lo = (int)n_lo;
+            p.n_hi = (int)n_hi;
+            p.ndeep = (int)ND;
+            const int64_t rest = NU - (int64_t)pd * n_lo;
+            const int64_t others = rest > 0 ? (rest + n_hi - 1) / n_hi : 0;
+            p.grid = (int)(pd + others < P ? pd + others : P);
+        }
+    }
+    if (!found) return false;
+    p.nunits = (int)NU;
+    p.mt = mt;
+    p.persist = true;
+    p.cnt_bytes = (size_t)nseq * H * kPersistSlices * sizeof(int32_t);
+    return true;
+}
+
 }  // namespace
+
+int device_sm_count() {
+    static int count[64];
+    static PerDeviceOnce once;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (per_device_once(once, [&] {
+            return cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+        }) != cudaSuccess)
+        return 0;
+    return count[dev];
+}
+
+size_t counter_bytes(const ripe_cache_s* c) {
+    return ((size_t)c->Bmax * c->H * kPersistSlices * sizeof(int32_t) + 255) / 256 * 256;
+}
 
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
                        bool capacity) {
@@ -402,6 +497,11 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
     p.a_ub = A_ub;
     p.win_ub = (len_ub < c->Wcap ? len_ub : c->Wcap) + max_ntok;
     p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
+    if (p.fused && all_depths && plan_persist(c, nbranch / c->R, max_ntok, len_ub, p)) {
+        p.part_bytes = verify_work_bytes(nrows, c->H, c->d, p.nsplit + 1);
+        p.work_bytes = counter_bytes(c) + p.part_bytes;
+        return p;
+    }
     int64_t ns;
     if (p.fused) {
         // One CTA per (sequence group, head, split); splits (a cluster, at most 8)
@@ -433,12 +533,14 @@ void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit
     int chunk = (A_ub + nsplit - 1) / nsplit;
     chunk = (chunk + align - 1) / align * align;
     p.chunk = chunk < align ? align : chunk;
-    p.work_bytes = verify_work_bytes(nrows, c->H, c->d, nsplit + 1);
+    p.cnt_bytes = 0;
+    p.part_bytes = verify_work_bytes(nrows, c->H, c->d, nsplit + 1);
+    p.work_bytes = counter_bytes(c) + p.part_bytes;
 }
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
                           const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,
-                          void* O, float* lse, void* work, cudaStream_t st) {
+                          void* O, float* lse, void* cnt, void* work, cudaStream_t st) {
     VerifyArgs a;
     a.s = store_view(c);
     a.ba = ba;
@@ -454,7 +556,13 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     a.part_o = reinterpret_cast<float*>(wb + verify_ml_bytes(ba.nrows, c->H, a.nseg));
     cudaError_t e;
     const int win_ub = plan.win_ub;
-    if (plan.fused) {
+    if (plan.persist) {
+        // The test hook is consumed by the launch it applies to.
+        const long long probe = const_cast<ripe_cache_s*>(c)->probe_cycles.exchange(0);
+        e = launch_persist(c->tmaps, a, reinterpret_cast<int32_t*>(cnt), plan.pd, plan.n_lo, plan.n_hi, plan.ndeep,
+                           plan.nunits, plan.grid, plan.mt, probe, ba.sliding, st);
+        if (e != cudaSuccess) return e;
+    } else if (plan.fused) {
         // The whole call in one kernel; programmatic dependent launch lets its
         // prologue overlap the tail of the previous kernel in the stream.
         e = launch_fused(c->tmaps, a, plan.gslots, plan.mt, true, st);

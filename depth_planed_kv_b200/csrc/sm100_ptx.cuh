@@ -49,13 +49,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Slow path of mbar_wait, out of line so that the many wait sites stay small.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* err) {
+// Slow path of mbar_wait, out of line so that the many wait sites stay small:
+// gives up after `limit` clock cycles (recording RIPE_DEVERR_TIMEOUT and setting
+// *abort) or as soon as *abort is set.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* err,
+                                                   long long limit = (1ll << 31)) {
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > (1ll << 31)) {
+        if (clock64() - t0 > limit) {
             *abort = 1;
             set_device_error(err, RIPE_DEVERR_TIMEOUT);
             return false;

@@ -64,11 +64,14 @@ _sig("ripe_evict", [_P, _P, _I, _P])
 _sig("ripe_truncate", [_P, _P, _P, _I, _P])
 _sig("ripe_verify_attn", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
 _sig("ripe_verify_attn_all_depths", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
+_sig("ripe_verify_attn_all_depths_sliding", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
 _sig("ripe_verify_attn_noalloc", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P,
                                   ctypes.POINTER(ctypes.c_size_t)])
 _sig("ripe_reserve_workspace", [_P, _I])
 _sig("ripe_synth_fill", [_P, _P, _P, _I, ctypes.c_uint64, _P, _P])
 _sig("ripe_cache_verify_path", [_P, ctypes.POINTER(_I)])
+_sig("ripe_debug_stall_next_verify", [_P, ctypes.c_longlong])
+_sig("ripe_accept", [_I, _I, _I, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P])
 _sig("ripe_cache_buffers", [_P] + [ctypes.POINTER(_P)] * 7)
 _sig("ripe_read_meta", [_P, _P, _P, _P, _P])
 _sig("ripe_get_device_error", [_P, _P, _P])
@@ -78,8 +81,8 @@ _sig("ripe_last_error", [], ctypes.c_char_p)
 
 EXPORTED = ["ripe_cache_bytes", "ripe_cache_create", "ripe_cache_destroy", "ripe_cache_reset",
             "ripe_append", "ripe_evict", "ripe_truncate", "ripe_verify_attn",
-            "ripe_verify_attn_all_depths", "ripe_verify_attn_noalloc", "ripe_reserve_workspace",
-            "ripe_synth_fill", "ripe_cache_verify_path",
+            "ripe_verify_attn_all_depths", "ripe_verify_attn_all_depths_sliding", "ripe_verify_attn_noalloc", "ripe_reserve_workspace",
+            "ripe_synth_fill", "ripe_cache_verify_path", "ripe_debug_stall_next_verify", "ripe_accept",
             "ripe_cache_buffers", "ripe_read_meta", "ripe_get_device_error", "ripe_launch_count",
             "ripe_error_string", "ripe_last_error"]
 
@@ -117,6 +120,22 @@ def _dtype_code(dtype: torch.dtype) -> int:
 
 def launch_count() -> int:
     return int(_lib.ripe_launch_count())
+
+
+def ripe_accept(zp: torch.Tensor, zq: torch.Tensor, zf: Optional[torch.Tensor], x1: torch.Tensor,
+                x2: Optional[torch.Tensor], u: torch.Tensor, temperature: float, stream=None):
+    """LoopSpec acceptance of [nseq][k] draft positions.  zp, zq, zf: float32
+    [nseq][k][V] logits (zf None: no fallback); x1, x2: int32 [nseq][k]; u: float32
+    [nseq][k][3].  Returns (n_accepted, token, path) as int32 [nseq] tensors."""
+    nseq, k, V = zp.shape
+    for t in (zp, zq) + ((zf,) if zf is not None else ()):
+        assert t.dtype == torch.float32 and t.is_contiguous() and t.shape == zp.shape
+    assert x1.dtype == torch.int32 and u.dtype == torch.float32 and u.shape == (nseq, k, 3)
+    out = [torch.empty(nseq, dtype=torch.int32, device=zp.device) for _ in range(3)]
+    _check(_lib.ripe_accept(nseq, k, V, _ptr(zp), _ptr(zq), _ptr(zf), _ptr(x1), _ptr(x2), _ptr(u),
+                            ctypes.c_float(temperature), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]),
+                            _stream(stream)), "ripe_accept")
+    return tuple(out)
 
 
 def ripe_cache_bytes(layers, R, H, d, W, Tmax, max_seqs, kmax, dtype=torch.bfloat16) -> int:
@@ -221,7 +240,23 @@ class RipeCache:
                                                 ctypes.c_float(scale), _ptr(O), _ptr(lse),
                                                 _stream(stream)), "ripe_verify_attn_all_depths")
 
+    def ripe_verify_attn_all_depths_sliding(self, layer: int, seq_ids: torch.Tensor, k: int, Q: torch.Tensor,
+                                            Kblk: torch.Tensor, Vblk: torch.Tensor, O: torch.Tensor,
+                                            lse: Optional[torch.Tensor] = None,
+                                            ctx_len: Optional[torch.Tensor] = None, scale: float = 0.0,
+                                            stream=None):
+        """The all-depths call under the per-query sliding window (same layouts)."""
+        _check(_lib.ripe_verify_attn_all_depths_sliding(self.handle, layer, _ptr(seq_ids), seq_ids.numel(), k,
+                                                        _ptr(Q), _ptr(Kblk), _ptr(Vblk), _ptr(ctx_len),
+                                                        ctypes.c_float(scale), _ptr(O), _ptr(lse),
+                                                        _stream(stream)), "ripe_verify_attn_all_depths_sliding")
+
     # --- inspection ------------------------------------------------------------
+    def ripe_debug_stall_next_verify(self, cycles: int):
+        """Test hook: the next persistent-kernel verify waits `cycles` on a barrier
+        nothing signals, so its bounded wait runs out (RIPE_DEVERR_TIMEOUT)."""
+        _check(_lib.ripe_debug_stall_next_verify(self.handle, int(cycles)), "ripe_debug_stall_next_verify")
+
     def ripe_cache_verify_path(self) -> int:
         """1: the fused sm_100a kernel serves verify; 0: the CUDA-core kernels."""
         out = ctypes.c_int()

@@ -215,6 +215,23 @@ int ripe_verify_attn_all_depths(ripe_cache_t cache, int layer, const int32_t* se
                                 ripe_stream_t stream);
 
 /*
+ * ripe_verify_attn_all_depths under the per-query sliding-window reading (the
+ * RIPE abstract's fifth sentence read per query): draft token j, at position
+ * T + j, reads the W most recent positions T+j-W+1 .. T+j at its own depth r --
+ * a committed one only while the store still holds its planes (p >= ws) -- and
+ * every older position at the deepest plane R; an older draft token j' < j-W+1 is
+ * read at plane R, which is its depth-R row in the same call.  With W >= k no
+ * draft token is read at plane R (batched verification is then block-independent).
+ * Same arguments and layouts as ripe_verify_attn_all_depths.  Served by the
+ * persistent sm_100a kernel only (bf16, d in {64, 96, 128}, k*R <= 256 and
+ * R*ceil(k/8) <= 64); RIPE_ERR_UNSUPPORTED otherwise.
+ */
+int ripe_verify_attn_all_depths_sliding(ripe_cache_t cache, int layer, const int32_t* seq_ids_dev, int nseq,
+                                        int k, const void* Q, const void* Kblk, const void* Vblk,
+                                        const int32_t* ctx_len_dev, float scale, void* O, float* lse,
+                                        ripe_stream_t stream);
+
+/*
  * ripe_verify_attn for callers that cannot allocate device memory.  The pages
  * have no counterpart: this is a deployment variant, not part of the method.
  *
@@ -272,6 +289,48 @@ int ripe_synth_fill(ripe_cache_t cache, const int32_t* seq_ids_host, const int32
  */
 enum { RIPE_PATH_CUDA_CORE = 0, RIPE_PATH_FUSED_SM100 = 1 };
 int ripe_cache_verify_path(ripe_cache_t cache, int* path);
+
+/*
+ * The acceptance step of self-speculative decoding, in LoopSpec's order (LoopSpec
+ * article, sections on the second branch and on the final check): for each draft
+ * position, first the early draft x1 is tested against the final distribution,
+ * then the fallback x2 prepared from a deeper state, and only after both are
+ * rejected the pipeline restarts from what the final distribution still has to
+ * give.  Sampling keeps the final distribution; greedy decoding (temperature 0)
+ * keeps the final argmax.
+ *   zp, zq, zf: device float [nseq][k][V] logits of the final loop, of the draft's
+ *       loop and of the deeper loop the fallback came from (zf NULL: no fallback).
+ *   x1, x2: device int32 [nseq][k] the draft and fallback tokens (x2 may be NULL
+ *       only without zf).
+ *   u: device float [nseq][k][3] uniforms in [0, 1): accept x1, accept x2, restart.
+ *   temperature >= 0 (0: greedy).
+ * With p, q1, qf the softmaxes at the temperature: x1 is accepted if
+ * u0 * q1(x1) < p(x1); the fallback exists if qf(x1) < q1(x1) at temperature 1 and
+ * q2 = norm((qf - q1)+) has mass; x2 is accepted if u1 * q2(x2) < p1(x2) with
+ * p1 = norm((p - q1)+); else the restart token is the smallest v whose running sum
+ * of norm((p1 - q2)+) (p1 without a fallback) exceeds u2 times its total.  A
+ * remainder without mass is replaced by the distribution it came from.  Positions
+ * are checked in order and the first rejected x1 ends the block.
+ * Outputs (device int32 [nseq]): n_accepted (drafts accepted, 0..k), token (the
+ * fallback or restart token emitted at position n_accepted, -1 when all k were
+ * accepted) and path (0 all accepted, 1 fallback accepted, 2 restart).
+ * fp32 arithmetic; one CTA per sequence.
+ */
+int ripe_accept(int nseq, int k, int V, const float* zp, const float* zq, const float* zf, const int32_t* x1,
+                const int32_t* x2, const float* u, float temperature, int32_t* n_accepted, int32_t* token,
+                int32_t* path, ripe_stream_t stream);
+
+/*
+ * Test hook for the bounded-wait error path (the pages have no counterpart).  The
+ * next all-depths verify on this cache that runs in the persistent sm_100a kernel
+ * makes its softmax warps first wait, at most `cycles` SM clock cycles (0 <= cycles
+ * <= 2^31; 0 turns the hook off), on a barrier that nothing signals.  The wait runs
+ * out, the kernel records RIPE_DEVERR_TIMEOUT, lets its copies and tensor-core
+ * operations in flight finish, and returns with that call's outputs incomplete;
+ * ripe_get_device_error then reports it and clears the merge counters, and later
+ * calls are exact again.  No fault, trap or unbounded wait is involved.
+ */
+int ripe_debug_stall_next_verify(ripe_cache_t cache, long long cycles);
 
 /* Device pointers of the store parts (tests compare them byte for byte); any
  * output may be NULL. */

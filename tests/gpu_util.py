@@ -57,3 +57,29 @@ def oracle_units(wl, layer, ctx, ws, branches, seq_sample, head_sample, mode=1):
     for (bi, b), t in zip(sel, table):
         out[bi] = (O[t[3]:t[3] + t[2]], lse[t[3]:t[3] + t[2]])
     return out
+
+
+def run_all_depths(cache, wl, layer, nseq, k, seqs=None, ctx_len=None, with_lse=True):
+    seqs = list(range(nseq)) if seqs is None else seqs
+    table, Q, Kb, Vb = all_depth_rows(wl, layer, nseq, seqs, k)
+    shape = (nseq, k, wl.R, wl.H, wl.d)
+    q, kb, vb = (to_dev(x.reshape(shape), wl) for x in (Q, Kb, Vb))
+    O = torch.full(shape, float("nan"), dtype=torch_dtype(wl), device="cuda")
+    lse = torch.full((nseq, k, wl.R, wl.H), float("nan"), device="cuda") if with_lse else None
+    ids = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+    cache.ripe_verify_attn_all_depths(layer, ids, k, q, kb, vb, O, lse, ctx_len=ctx_len)
+    torch.cuda.synchronize()
+    O = O.float().cpu().numpy().reshape(nseq * k * wl.R, wl.H, wl.d)
+    lse = lse.cpu().numpy().reshape(nseq * k * wl.R, wl.H) if with_lse else None
+    return table, O, lse, (Q, Kb, Vb)
+
+
+def oracle_all_depths(wl, layer, nseq, k, T, ws, seqs=None, heads=None, mode=1):
+    seqs = list(range(nseq)) if seqs is None else seqs
+    views = [seq_planes(wl, layer, s, T[i], ws[i], heads=heads) for i, s in enumerate(seqs)]
+    table, Q, Kb, Vb = all_depth_rows(wl, layer, nseq, seqs, k, heads=heads)
+    return OR.verify(views, table, Q, Kb, Vb, 1 / math.sqrt(wl.d), mode)
+
+
+def check_lse(got, ref):
+    assert np.abs(got - ref).max() < 2e-3, np.abs(got - ref).max()
