@@ -50,7 +50,7 @@ bool stream_capturing(cudaStream_t st) {
 namespace {
 
 struct Layout {
-    size_t kdeep, vdeep, kwin, vwin, len, ws, rfloor, err, total;
+    size_t kdeep, vdeep, kwin, vwin, len, ws, rfloor, base, fpos, err, total;
 };
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -84,7 +84,9 @@ Layout layout_of(int L, int R, int H, int d, int W, int Tmax, int Bmax, int kmax
     y.len = y.vwin + ring;
     y.ws = y.len + round256(sizeof(int32_t) * Bmax);
     y.rfloor = y.ws + round256(sizeof(int32_t) * Bmax);
-    y.err = y.rfloor + round256(sizeof(int32_t) * Bmax);
+    y.base = y.rfloor + round256(sizeof(int32_t) * Bmax);
+    y.fpos = y.base + round256(sizeof(int32_t) * Bmax);
+    y.err = y.fpos + round256(sizeof(int32_t) * Bmax);
     y.total = y.err + 256;
     return y;
 }
@@ -236,6 +238,8 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
     c->kwin = c->base + y.kwin; c->vwin = c->base + y.vwin;
     c->len = (int32_t*)(c->base + y.len); c->ws = (int32_t*)(c->base + y.ws);
     c->rfloor = (int32_t*)(c->base + y.rfloor);
+    c->fbase = (int32_t*)(c->base + y.base);
+    c->fpos = (int32_t*)(c->base + y.fpos);
     c->err = (int32_t*)(c->base + y.err);
     c->tc_ready = false;
     if (fused_supported(dtype, d)) {
@@ -245,8 +249,10 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
             fail(RIPE_OK, "tensor maps of this store cannot be built (code %d); verify uses the CUDA-core "
                  "kernels (ripe_cache_verify_path reports 0)", tm);
     }
-    // Zeroed store: key tiles that overrun a region read finite values.
+    // Zeroed store: key tiles that overrun a region read finite values.  Every
+    // sequence starts as the owner of its own deep plane (not a fork).
     cudaError_t e = cudaMemset(c->base, 0, y.total);
+    if (e == cudaSuccess) e = launch_init_meta(c, nullptr);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         if (c->owns) cudaFree(c->base);
@@ -303,6 +309,16 @@ int ripe_evict(ripe_cache_t c, const int32_t* seq_ids, int nseq, ripe_stream_t s
     if (!seq_ids) return fail(RIPE_ERR_INVALID_ARG, "seq_ids is NULL");
     cudaError_t e = launch_evict(c, seq_ids, nseq, as_stream(stream));
     return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "evict launch");
+}
+
+int ripe_fork(ripe_cache_t c, const int32_t* parent_ids, const int32_t* child_ids, int nseq, ripe_stream_t stream) {
+    int rc = check_cache(c);
+    if (rc != RIPE_OK) return rc;
+    if (nseq < 0 || nseq > c->Bmax) return fail(RIPE_ERR_INVALID_ARG, "nseq=%d outside [0,%d]", nseq, c->Bmax);
+    if (nseq == 0) return RIPE_OK;
+    if (!parent_ids || !child_ids) return fail(RIPE_ERR_INVALID_ARG, "NULL pointer argument");
+    cudaError_t e = launch_fork(c, parent_ids, child_ids, nseq, as_stream(stream));
+    return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "fork launch");
 }
 
 int ripe_truncate(ripe_cache_t c, const int32_t* seq_ids, const int32_t* new_len, int nseq,
@@ -450,6 +466,19 @@ int ripe_cache_buffers(ripe_cache_t c, void** kdeep, void** vdeep, void** kwin, 
     if (ws) *ws = c->ws;
     if (rfloor) *rfloor = c->rfloor;
     return RIPE_OK;
+}
+
+int ripe_read_forks(ripe_cache_t c, int32_t* fbase_host, int32_t* fpos_host, ripe_stream_t stream) {
+    int rc = check_cache(c);
+    if (rc != RIPE_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    cudaError_t e = cudaSuccess;
+    if (fbase_host)
+        e = cudaMemcpyAsync(fbase_host, c->fbase, sizeof(int32_t) * c->Bmax, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && fpos_host)
+        e = cudaMemcpyAsync(fpos_host, c->fpos, sizeof(int32_t) * c->Bmax, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "read_forks");
 }
 
 int ripe_read_meta(ripe_cache_t c, int32_t* len_host, int32_t* ws_host, int32_t* rfloor_host,

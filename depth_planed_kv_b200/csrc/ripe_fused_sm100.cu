@@ -67,6 +67,7 @@ struct BranchEnt {
 
 struct GroupInfo {
     int first, nb, seq, nrows, T, A, key_begin, key_end, units;
+    int fb, fp;  // deep positions below fp are read from sequence fb (a fork's parent)
 };
 
 template <int D, int MT, int ST, int NW, int NS>
@@ -419,10 +420,12 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
             ubase += __shfl_sync(0xffffffffu, uincl, 31);
         }
         if (lane == 0) {
-            GroupInfo info{first, nb, seq, base, 0, 0, 0, 0, ubase};
+            GroupInfo info{first, nb, seq, base, 0, 0, 0, 0, ubase, seq, 0};
             if (seq >= 0 && base > 0) {
                 info.T = context_length(s.len, a.ctx, s.err, seq, split == 0 && h == 0);
                 info.A = min(s.ws[seq], info.T);
+                info.fp = s.fpos[seq];
+                info.fb = info.fp > 0 ? s.fbase[seq] : seq;
                 info.key_begin = split * a.chunk;
                 info.key_end = min(info.A, info.key_begin + a.chunk);
             } else {
@@ -448,13 +451,16 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
             if (warp == 4) {
                 // ------------------------------------------------ TMA producer
                 if (lane == 0) {
-                    const int row_base = ((a.layer * s.Bmax + G.seq) * s.H + h) * s.Tmax + G.key_begin;
+                    // A fork's tiles below its fork position (a multiple of the tile) come from
+                    // its parent's deep plane.
+                    const int own_base = ((a.layer * s.Bmax + G.seq) * s.H + h) * s.Tmax + G.key_begin;
+                    const int par_base = ((a.layer * s.Bmax + G.fb) * s.H + h) * s.Tmax + G.key_begin;
                     int issued = 0;
                     for (int it = 0; it < total_it; ++it) {
                         const int i = it % ntiles, st = it % ST;
                         if (it >= ST && !mbar_wait(kv_empty + st, ((it / ST) - 1) & 1, abort_flag, s.err)) break;
                         issued = it + 1;
-                        const int y = row_base + i * kN;
+                        const int y = (G.key_begin + i * kN < G.fp ? par_base : own_base) + i * kN;
                         mbar_expect_tx(k_full + st, Lay::KV_STAGE);
 #pragma unroll
                         for (int c = 0; c < NCH; ++c)
@@ -775,6 +781,7 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
         // first window row of plane R.
         const int ring_y0 = ((a.layer * s.Bmax + G.seq) * s.H + h) * (s.R - 1) * s.Wcap;
         const int deep_y0 = ((a.layer * s.Bmax + G.seq) * s.H + h) * s.Tmax + G.A;
+        const int deep_yp0 = ((a.layer * s.Bmax + G.fb) * s.H + h) * s.Tmax + G.A;  // fork parent
         const int q4 = lane & 3, r8 = lane >> 2;
         if (lane == 0) {
             prefetch_tmap(&tm.wk);
@@ -804,9 +811,12 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                 uint64_t* bar = wbar + stage;
                 const bool ring = w.depth < s.R;
                 const int k0t = t * kWinKeys;
-                if (k0t + kWinKeys <= w.wk) {
+                // deep rows of a tile on one side of a fork position come from one plane
+                const bool one_owner = ring || ((G.A + k0t < G.fp) == (G.A + k0t + kWinKeys - 1 < G.fp));
+                if (k0t + kWinKeys <= w.wk && one_owner) {
                     if (lane == 0) {
-                        const int y = (ring ? ring_y0 + (w.depth - 1) * s.Wcap + w.lo : deep_y0) + k0t;
+                        const int y = (ring ? ring_y0 + (w.depth - 1) * s.Wcap + w.lo
+                                            : (G.A + k0t < G.fp ? deep_yp0 : deep_y0)) + k0t;
                         const CUtensorMap* mk = ring ? &tm.wk : &tm.rk;
                         const CUtensorMap* mv = ring ? &tm.wv : &tm.rv;
                         fence_proxy_async_smem();  // earlier reads of this stage come first
@@ -832,7 +842,8 @@ verify_kernel(const __grid_constant__ TMaps tm, VerifyArgs a) {
                     bool ok;
                     if (key < w.wk) {
                         ok = win_valid(w, wkeys, s.R, s.Wcap, key);
-                        const int64_t off = wbase + (int64_t)key * 2 * D + q4 * 16;
+                        const int64_t off = (!ring && G.A + key < G.fp ? deep_row(s, a.layer, G.fb, h, G.A) : wbase) +
+                                            (int64_t)key * 2 * D + q4 * 16;
                         if (ok) {
                             kp = (ring ? s.kwin : s.kdeep) + off;
                             vp = (ring ? s.vwin : s.vdeep) + off;
@@ -1154,12 +1165,12 @@ cudaError_t launch_fused(const void* tmaps, const VerifyArgs& args, int gslots, 
 // the kernels' shared-memory layouts expect.  Deep planes (rows = L*Bmax*H*Tmax)
 // in 64-row boxes (deep region) and 16-row boxes (window tiles at depth R); ring
 // planes (rows = L*Bmax*H*(R-1)*Wcap) in 16-row boxes; ring and deep planes again
-// in 8-row boxes for the persistent kernel.  Rows past the end of a view read as
-// zeros.
+// in 8-row boxes and in Wcap-row boxes for the persistent kernel.  Rows past the
+// end of a view read as zeros.
 int make_tensor_maps(ripe_cache_s* c) {
     const EncodeFn encode = encode_fn();
     if (!encode) return -1;
-    static_assert(sizeof(c->tmaps) == 10 * sizeof(CUtensorMap), "tensor map bundle");
+    static_assert(sizeof(c->tmaps) == 14 * sizeof(CUtensorMap), "tensor map bundle");
     const cuuint64_t deep_rows = (cuuint64_t)c->L * c->Bmax * c->H * c->Tmax;
     const cuuint64_t ring_rows = (cuuint64_t)c->L * c->Bmax * c->H * (c->R - 1) * c->Wcap;
     if (deep_rows >= (1ull << 31) || ring_rows >= (1ull << 31)) return -2;
@@ -1172,7 +1183,10 @@ int make_tensor_maps(ripe_cache_s* c) {
     };
     // With no ring planes (R = 1) the ring maps are never used; they alias the deep planes.
     const bool ring = ring_rows > 0;
-    const Spec spec[10] = {{c->kdeep, deep_rows, (cuuint32_t)kN},
+    // A whole ring plane (Wcap rows) per box when that fits a box (<= 256 rows).
+    c->full_box = c->Wcap <= 256;
+    const cuuint32_t full_rows = (cuuint32_t)(c->full_box ? c->Wcap : 256);
+    const Spec spec[14] = {{c->kdeep, deep_rows, (cuuint32_t)kN},
                            {c->vdeep, deep_rows, (cuuint32_t)kN},
                            {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
                            {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, (cuuint32_t)kWinKeys},
@@ -1181,8 +1195,12 @@ int make_tensor_maps(ripe_cache_s* c) {
                            {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, 8u},
                            {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, 8u},
                            {c->kdeep, deep_rows, 8u},
-                           {c->vdeep, deep_rows, 8u}};
-    for (int i = 0; i < 10; ++i) {
+                           {c->vdeep, deep_rows, 8u},
+                           {ring ? c->kwin : c->kdeep, ring ? ring_rows : deep_rows, full_rows},
+                           {ring ? c->vwin : c->vdeep, ring ? ring_rows : deep_rows, full_rows},
+                           {c->kdeep, deep_rows, full_rows},
+                           {c->vdeep, deep_rows, full_rows}};
+    for (int i = 0; i < 14; ++i) {
         const cuuint64_t dims[2] = {(cuuint64_t)c->d, spec[i].rows};
         const cuuint32_t box[2] = {32, spec[i].box_rows};
         CUresult r = encode(reinterpret_cast<CUtensorMap*>(c->tmaps[i]), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,

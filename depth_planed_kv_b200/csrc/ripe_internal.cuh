@@ -18,7 +18,7 @@ struct ripe_cache_s {
     bool owns;
     char* base;
     char *kdeep, *vdeep, *kwin, *vwin;
-    int32_t *len, *ws, *rfloor, *err;
+    int32_t *len, *ws, *rfloor, *fbase, *fpos, *err;
     // Host-side upper bound of len over all sequences (grows with append/fill);
     // sizes the deep-region split grid without reading device metadata.
     int len_ub;
@@ -29,8 +29,10 @@ struct ripe_cache_s {
     // (bf16, d in {64, 96, 128}): deep K, V planes in 64-row boxes (deep region),
     // ring K, V planes and deep K, V planes in 16-row boxes (window tiles of the
     // cluster kernel), and the same four in 8-row boxes (window chunks of the
-    // persistent kernel).
-    alignas(64) unsigned char tmaps[10][128];
+    // persistent kernel), and ring and deep planes in boxes of Wcap rows (a whole
+    // ring plane in one box; only when Wcap <= 256, see full_box).
+    alignas(64) unsigned char tmaps[14][128];
+    bool full_box;
     bool tc_ready;
     // Test hook (ripe_debug_stall_next_verify): clock cycles of a wait that nothing
     // ends, taken by the next persistent-kernel verify; 0 = off.
@@ -41,15 +43,17 @@ struct ripe_cache_s {
 struct StoreView {
     char *kdeep, *vdeep, *kwin, *vwin;
     // len: committed length; ws: window start; rfloor: lowest position whose ring
-    // slots still hold its own planes (ws >= rfloor; evict leaves it alone).
-    int32_t *len, *ws, *rfloor, *err;
+    // slots still hold its own planes (ws >= rfloor; evict leaves it alone);
+    // fbase, fpos: a fork reads its deep positions below fpos from sequence fbase
+    // (fbase = itself and fpos = 0 for a sequence that is not a fork).
+    int32_t *len, *ws, *rfloor, *fbase, *fpos, *err;
     int L, R, H, d, Tmax, Bmax, Wcap, W, esize;
 };
 
 static inline StoreView store_view(const ripe_cache_s* c) {
     StoreView s;
     s.kdeep = c->kdeep; s.vdeep = c->vdeep; s.kwin = c->kwin; s.vwin = c->vwin;
-    s.len = c->len; s.ws = c->ws; s.rfloor = c->rfloor; s.err = c->err;
+    s.len = c->len; s.ws = c->ws; s.rfloor = c->rfloor; s.fbase = c->fbase; s.fpos = c->fpos; s.err = c->err;
     s.L = c->L; s.R = c->R; s.H = c->H; s.d = c->d; s.Tmax = c->Tmax; s.Bmax = c->Bmax;
     s.Wcap = c->Wcap; s.W = c->W; s.esize = c->esize;
     return s;
@@ -58,6 +62,12 @@ static inline StoreView store_view(const ripe_cache_s* c) {
 // Byte offset of row (layer, seq, head, position) of the deep plane.
 __host__ __device__ inline int64_t deep_row(const StoreView& s, int l, int b, int h, int64_t p) {
     return ((((int64_t)l * s.Bmax + b) * s.H + h) * s.Tmax + p) * (int64_t)s.d * s.esize;
+}
+
+// The sequence whose deep plane holds position p of sequence b (its fork parent
+// below the fork position, else b itself).
+__device__ __forceinline__ int deep_owner(const StoreView& s, int b, int64_t p) {
+    return p < s.fpos[b] ? s.fbase[b] : b;
 }
 
 // Byte offset of ring slot `slot` of plane r (1..R-1).

@@ -13,6 +13,9 @@ cudaError_t launch_evict(const ripe_cache_s* c, const int32_t* seq_ids, int nseq
 cudaError_t launch_reset(const ripe_cache_s* c, const int32_t* seq_ids, int nseq, cudaStream_t st);
 cudaError_t launch_truncate(const ripe_cache_s* c, const int32_t* seq_ids, const int32_t* new_len, int nseq,
                             cudaStream_t st);
+cudaError_t launch_init_meta(const ripe_cache_s* c, cudaStream_t st);
+cudaError_t launch_fork(const ripe_cache_s* c, const int32_t* parents, const int32_t* children, int nseq,
+                        cudaStream_t st);
 cudaError_t launch_synth_fill(const ripe_cache_s* c, int b, int T, uint64_t seed, const float* coef,
                               cudaStream_t st);
 
@@ -57,10 +60,12 @@ bool fused_supported(int dtype, int d);
 cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int mt, bool pdl, cudaStream_t st);
 cudaError_t launch_persist(const void* tmaps, const VerifyArgs& a, int32_t* cnt, int pd, int n_lo, int n_hi,
                            int ndeep, int nunits, int grid, int mt, long long probe_cycles, int sliding,
-                           cudaStream_t st);
+                           int full_box, cudaStream_t st);
 // Window warps of a deep CTA and of another CTA of the persistent kernel (0: no kernel).
 void persist_shape(int d, int mt, int* nww_deep, int* nww_other);
-// The ten tensor maps of the sm_100a kernels (0 on success).
+// The persistent kernel's window units go through its stage ring (one producer warp).
+bool persist_ring_ok(int d, int mt, int Wcap, int k, int sliding, int full_box);
+// The fourteen tensor maps of the sm_100a kernels (0 on success).
 int make_tensor_maps(ripe_cache_s* c);
 // A tensor map of this call's Q as [rows][H][d], 128-row boxes of one head (false: none).
 struct CUtensorMap_st;

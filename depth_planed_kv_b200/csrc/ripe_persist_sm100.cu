@@ -55,10 +55,11 @@ constexpr int kMaxUnitsPerGroup = kPersistSlices;
 // one head.  All 32 columns wide with the 64-byte swizzle.
 struct PMaps {
     CUtensorMap dk, dv, wk, wv, rk, rv, q;
+    CUtensorMap wkf, wvf, rkf, rvf;  // ring / deep planes in boxes of Wcap rows (a whole ring plane)
 };
 
 struct DeepItem {
-    int g, h, c, seq, kb, ke, E, ntiles;
+    int g, h, c, seq, kb, ke, E, ntiles, fb, fp;  // fb, fp: fork parent and position
 };
 
 // Scalars of a launch beyond the common verify arguments.
@@ -76,6 +77,7 @@ struct PArgs {
     // draft token j at position T + j reads positions T+j-W+1 .. T+j at its own
     // depth, older ones at plane R; 0 = the store's window for every row.
     int sliding;
+    int full_box;  // the Wcap-row maps are valid (Wcap <= 256)
 };
 
 template <int D, int MT, int ST, int NWW, int KC>
@@ -100,11 +102,17 @@ struct PLayout {
     static constexpr int OFF_BAR = OFF_OST + OST_BYTES;
     // q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain, epi_done, probe
     static constexpr int NBAR = 1 + 3 * ST + 9;
-    static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;  // one per warp (window stage)
-    static constexpr int OFF_MISC = OFF_WBAR + NWARPS * 8;
+    // Window stage barriers: one per warp (full), then one per warp (empty, stage ring).
+    static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_MISC = OFF_WBAR + 2 * NWARPS * 8;
     static constexpr int OFF_ITEMS = OFF_MISC + 64;
     static constexpr int OFF_FLAGS = OFF_ITEMS + kMaxItems * (int)sizeof(DeepItem);
-    static constexpr int BYTES = OFF_FLAGS + 2 * kMaxUnitsPerGroup;
+    // Stage ring: the unit held by each stage.
+    static constexpr int DESC_BYTES = 96;
+    static constexpr int OFF_DESC = (OFF_FLAGS + 2 * kMaxUnitsPerGroup + 15) / 16 * 16;
+    // Stage ring: the ticket last issued into each stage.
+    static constexpr int OFF_ISS = OFF_DESC + NWARPS * DESC_BYTES;
+    static constexpr int BYTES = OFF_ISS + NWARPS * 4;
     static constexpr int SMEM = BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
@@ -128,11 +136,21 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
     return v;
 }
 
+// Arrival on a slice counter: release (this thread's earlier writes, and those of
+// the threads it synchronised with at a barrier, are visible to whoever acquires
+// the counter later) and acquire (the partials of earlier arrivals are visible to
+// this thread, and through a later barrier to its CTA).  Returns the old count.
+__device__ __forceinline__ int arrive_acq_rel(int32_t* p) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old;
+}
+
 // Context of sequence slot g of an all-depths call: its id, committed length T,
 // deep-region length A and the arrivals E each of its slices expects; ok is
 // false for an id outside the store (reported once).
 struct GroupCtx {
-    int seq, T, A, E;
+    int seq, T, A, E, fb, fp;  // fb, fp: deep positions below fp are read from sequence fb
     bool ok;
 };
 
@@ -144,26 +162,28 @@ __device__ __forceinline__ GroupCtx group_ctx(const VerifyArgs& a, int g, bool r
         if (report) set_device_error(a.s.err, RIPE_DEVERR_SEQ_RANGE);
         c.T = c.A = 0;
         c.E = 1;
+        c.fb = c.fp = 0;
         return c;
     }
     c.T = context_length(a.s.len, a.ctx, a.s.err, c.seq, report);
     c.A = min(a.s.ws[c.seq], c.T);
     c.E = deep_splits_used(c.A, a.chunk, a.nsplit) + 1;
+    c.fp = a.s.fpos[c.seq];
+    c.fb = c.fp > 0 ? a.s.fbase[c.seq] : c.seq;
     return c;
 }
 
-// Visibility of a window unit's key kk to row (token) j under the sliding window:
-// keys [0, nw) are window positions A + kk at plane r, [nw, nw + nblk) draft
-// tokens at plane r, then ndw window positions at plane R, then draft tokens at
-// plane R.  sbase = T - W + 1 - A is row 0's first plane-r position, minus A.
-__device__ __forceinline__ bool slide_visible(int kk, int j, int nw, int nblk, int ndw, int nk, int sbase, int W) {
-    if (kk < nw) return kk >= sbase + j;
-    if (kk < nw + nblk) {
-        const int jj = kk - nw;
-        return jj <= j && jj >= j - W + 1;
-    }
-    if (kk < nw + nblk + ndw) return kk - nw - nblk < sbase + j;
-    if (kk < nk) return kk - nw - nblk - ndw < j - W + 1;
+// Visibility to row (token) j, under the sliding window, of a window unit's key
+// that follows its window keys: e counts from the first such key; nblk draft
+// tokens at plane r, then ndw window positions A + e at plane R, then nbr draft
+// tokens at plane R.  sbase = T - W + 1 - A is row 0's first plane-r position,
+// minus A.
+__device__ __forceinline__ bool slide_visible(int e, int j, int nblk, int ndw, int nbr, int sbase, int W) {
+    if (e < nblk) return e <= j && e >= j - W + 1;        // draft token e at plane r
+    e -= nblk;
+    if (e < ndw) return e < sbase + j;                    // window position A + e at plane R
+    e -= ndw;
+    if (e < nbr) return e < j - W + 1;                    // draft token e at plane R
     return false;
 }
 
@@ -173,7 +193,7 @@ __device__ __forceinline__ int32_t* slice_counter(const VerifyArgs& a, const PAr
     return p.cnt + ((int64_t)g * a.s.H + h) * kPersistSlices + (r - 1) * QS + j / kWR;
 }
 
-template <int D, int MT, int ST, int NWW, int KC>
+template <int D, int MT, int ST, int NWW, int KC, bool RING>
 __global__ void __launch_bounds__(PLayout<D, MT, ST, NWW, KC>::THREADS, 1)
 persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     using Lay = PLayout<D, MT, ST, NWW, KC>;
@@ -206,6 +226,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     // a named barrier, read by all four after it, so that they decide alike even if
     // another role sets the flag in between.
     volatile int* stop_snap = reinterpret_cast<volatile int*>(sm + Lay::OFF_MISC + 12);
+    // Next window unit of this CTA's range to hand to a warp that asks for one.
+    int* unit_next = reinterpret_cast<int*>(sm + Lay::OFF_MISC + 16);
     DeepItem* items = reinterpret_cast<DeepItem*>(sm + Lay::OFF_ITEMS);
     uint8_t* known_last = sm + Lay::OFF_FLAGS;
     uint8_t* is_last = known_last + kMaxUnitsPerGroup;
@@ -235,9 +257,18 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             mbar_init(epi_done, 4);
             mbar_init(probe, 1);
         }
-        // Window stages: 32 cp.async arrivals (one per lane) + lane 0's expect_tx.
-        for (int i = 0; i < Lay::NWARPS; ++i) mbar_init(wbar + i, 33);
+        // Window stages: 32 cp.async arrivals (one per lane) + lane 0's expect_tx;
+        // the ring's empty barriers: one consumer's arrival.
+        for (int i = 0; i < Lay::NWARPS; ++i) {
+            mbar_init(wbar + i, 33);
+            mbar_init(wbar + Lay::NWARPS + i, 1);
+        }
+        *reinterpret_cast<int*>(sm + Lay::OFF_MISC + 20) = 0;  // the ring's next ticket
+        for (int i = 0; i < Lay::NWARPS; ++i) reinterpret_cast<int*>(sm + Lay::OFF_ISS)[i] = -1;
         *abort_flag = 0;
+        const int64_t ub = cta < pa.pd ? (int64_t)cta * pa.n_lo
+                                       : (int64_t)pa.pd * pa.n_lo + (int64_t)(cta - pa.pd) * pa.n_hi;
+        *unit_next = (int)(ub < pa.nunits ? ub : pa.nunits);
         fence_barrier_init();
     }
     if (deep_cta && warp == 5) {
@@ -271,6 +302,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             const GroupCtx gc = group_ctx(a, it.g, it.h == 0 && it.c == 0);
             it.seq = gc.seq;
             it.E = gc.E;
+            it.fb = gc.fb;
+            it.fp = gc.fp;
             // The last chunk takes every key past the others, so any deep length is
             // covered whatever the length the host planned for.
             it.kb = it.c * a.chunk;
@@ -294,14 +327,17 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 bool ok = true;
                 for (int n = 0; n < n_items && ok; ++n) {
                     const DeepItem& di = items[n];
-                    const int row_base = ((a.layer * s.Bmax + di.seq) * H + di.h) * s.Tmax + di.kb;
+                    // A fork's tiles below its fork position (a multiple of the tile) come
+                    // from its parent's deep plane.
+                    const int own_base = ((a.layer * s.Bmax + di.seq) * H + di.h) * s.Tmax + di.kb;
+                    const int par_base = ((a.layer * s.Bmax + di.fb) * H + di.h) * s.Tmax + di.kb;
                     for (int i = 0; i < di.ntiles; ++i, ++it) {
                         const int st = it % ST;
                         if (it >= ST && !mbar_wait(kv_empty + st, ((it / ST) - 1) & 1, abort_flag, s.err)) {
                             ok = false;
                             break;
                         }
-                        const int y = row_base + i * kN;
+                        const int y = (di.kb + i * kN < di.fp ? par_base : own_base) + i * kN;
                         mbar_expect_tx(k_full + st, Lay::KV_STAGE);
 #pragma unroll
                         for (int c = 0; c < NCH; ++c)
@@ -573,7 +609,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                         }
                     }
                 }
-                __threadfence();
+                // The barrier orders every softmax thread's partial writes before the
+                // arrivals; each arrival releases them and acquires the earlier ones.
                 if (t == 0) *stop_snap = *abort_flag;
                 softmax_bar();
                 const bool all_ok = !*stop_snap;
@@ -583,12 +620,11 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     bool last = false;
                     if (all_ok) {
                         last = known_last[u];
-                        if (!last) last = atomicAdd(cp, 1) == di.E - 1;
+                        if (!last) last = arrive_acq_rel(cp) == di.E - 1;
                         if (last) *cp = 0;  // the last arrival: nothing else touches it in this call
                     }
                     is_last[u] = last;
                 }
-                __threadfence();
                 softmax_bar();
                 // Merge the rows of the slices that ended here: this chunk's partial from
                 // TMEM and registers, the other deep chunks' and the window's from scratch.
@@ -665,21 +701,38 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     }
 
     // ======================================================== window units
-    // Deep CTA: warps 6.. with stages after the deep ones.  Other CTAs: every warp
-    // with a stage anywhere in the stage region.
-    const int wbase = deep_cta ? kDeepWarps : 0;
-    const int nww = deep_cta ? NWW : Lay::NW_FULL;
-    const int wi = warp - wbase;
-    if (wi >= 0 && wi < nww) {
-        uint8_t* stage = sm + (deep_cta ? Lay::OFF_W + wi * Lay::WSTAGE : wi * Lay::WSTAGE);
+    // Two forms (a template parameter).
+    // Per-warp stages: deep CTA: warps 6.. start at once with the stages after the
+    // deep ones; once the deep items are done (every deep warp at the named barrier
+    // below, so no copy or tensor-core read of the deep stages is in flight) the
+    // first deep warps join, with stages in the deep region.  Other CTAs: every warp
+    // with a stage anywhere in the stage region.  Warps take the CTA's units one at
+    // a time from a shared counter.  Each runs a unit one chunk of keys at a time
+    // through its own stage; when a unit's last chunk has been read out of the
+    // stage, the warp issues the next unit's first chunk and its Q loads, publishes
+    // the unit's partial and arrives, and looks at whether that arrival was the last
+    // only when the next unit ends (with the unit after it in flight), so that the
+    // round trips overlap.
+    // Stage ring (every unit one chunk, its queries in the chunk's last 8 key rows):
+    // one producer warp (the first window warp) walks the CTA's units in order and
+    // loads each into the next free stage of a ring; every other warp (the deep
+    // warps too, once their items are done) is a consumer that takes the next
+    // ticket, waits for that stage, computes, frees the stage at once and only then
+    // publishes and arrives.  The loads run ahead of the arrivals' round trips.
+    constexpr int NX = Lay::OFF_W / Lay::WSTAGE < kDeepWarps ? Lay::OFF_W / Lay::WSTAGE : kDeepWarps;
+    if (deep_cta && warp < kDeepWarps) asm volatile("bar.sync 2, %0;" ::"n"(32 * kDeepWarps) : "memory");
+    const int wfirst = deep_cta ? kDeepWarps : 0;  // the ring's producer
+    const bool win_role = RING ? true : deep_cta ? (warp >= kDeepWarps || warp < NX) : warp < Lay::NW_FULL;
+    if (win_role) {
+        uint8_t* stage = sm + (deep_cta && warp >= kDeepWarps ? Lay::OFF_W + (warp - kDeepWarps) * Lay::WSTAGE
+                                                              : warp * Lay::WSTAGE);
         uint64_t* bar = wbar + warp;
         const uint32_t stage_a = smem_u32(stage);
         const int64_t ub64 = cta < pa.pd ? (int64_t)cta * pa.n_lo
                                          : (int64_t)pa.pd * pa.n_lo + (int64_t)(cta - pa.pd) * pa.n_hi;
         const int64_t ue64 = ub64 + (cta < pa.pd ? pa.n_lo : pa.n_hi);
-        const int ubeg = (int)(ub64 < pa.nunits ? ub64 : pa.nunits);
         const int uend = (int)(ue64 < pa.nunits ? ue64 : pa.nunits);
-        constexpr int NKS = D / 16, NMT = D / 16, NT = KC / 16;
+        constexpr int NKS = D / 16, NMT = D / 16, NT = KC / 16, VPR = NCH * 4;
         const float c2 = a.scale_log2;
         const int q4 = lane & 3, r8 = lane >> 2;
         const int ra = 2 * q4, rb = ra + 1;
@@ -692,178 +745,348 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
         const uint32_t v_sw1 = ((((lane >> 3) & 1) + 2) ^ ((rv >> 1) & 3)) << 4;
         int cached_g = -1;
         GroupCtx gc{};
-        uint32_t phase = 0;
-        bool wok = true;
-        for (int u = ubeg + wi; u < uend && wok; u += nww) {
+
+        // A unit (group g, head h, depth r, slice j0..j0+nr-1) and its keys: nw window
+        // positions A.. at plane r (ring) or R (deep rows), nblk draft tokens at plane
+        // r, and under the sliding window ndw window positions and nbr draft tokens at
+        // plane R.
+        // Whole-window units (fast): when the ring plane (Wcap slots) and the unit's
+        // other keys fit one chunk, the window keys are the Wcap ring slots in slot
+        // order (or Wcap deep rows from A at depth R), loaded by one Wcap-row TMA box
+        // per column chunk; koff = Wcap keys then precede the draft tokens.
+        // Otherwise koff = nw window keys in position order, 8-row boxes.
+        struct Unit {
+            int g, h, r, j0, nr, nw, nblk, ndw, nbr, nk, koff, slot0, sbase, E, A, seq, fb, fp;
+            bool ring, slide, ok, fast;
+        };
+        // What the merge of a unit's slice needs.
+        struct Slice {
+            int g, h, r, j0, nr, E;
+        };
+        auto describe = [&](int u) {
+            Unit w;
             const int q = u % QS;
-            const int r = (u / QS) % R + 1;
-            const int h = (u / (QS * R)) % H;
-            const int g = u / (QS * R * H);
-            if (g != cached_g) {
-                gc = group_ctx(a, g, false);
-                cached_g = g;
+            w.r = (u / QS) % R + 1;
+            w.h = (u / (QS * R)) % H;
+            w.g = u / (QS * R * H);
+            if (w.g != cached_g) {
+                gc = group_ctx(a, w.g, false);
+                cached_g = w.g;
             }
-            if (!gc.ok) continue;
-            const int j0 = q * kWR, nr = min(kWR, k - j0);
-            const int nw = gc.T - gc.A, nblk = j0 + nr;
-            const bool ring = r < R;
+            w.ok = gc.ok;
+            w.E = gc.E;
+            w.A = gc.A;
+            w.seq = gc.seq;
+            w.j0 = q * kWR;
+            w.nr = min(kWR, k - w.j0);
+            w.nw = gc.T - gc.A;
+            w.nblk = w.j0 + w.nr;
+            w.ring = w.r < R;
             // Sliding window (depth r < R only; at depth R both readings agree): row j
             // reads window position p at plane r iff p >= T + j - W + 1, else at plane
-            // R, and draft token j' at plane r iff j' >= j - W + 1, else its depth-R
-            // row.  The unit's keys then continue with plane-R copies of the first
-            // window positions (ndw) and the depth-R rows of the first draft tokens
-            // (nbr), each masked per row.
-            const bool slide = pa.sliding && ring;
-            const int sbase = gc.T - s.W + 1 - gc.A;  // (T + j - W + 1) - A at j = 0
-            const int ndw = slide ? max(0, min(nw, sbase + j0 + nr - 1)) : 0;
-            const int nbr = slide ? max(0, j0 + nr - s.W) : 0;
-            const int nk = nw + nblk + ndw + nbr;
-            const int slot0 = gc.A % s.Wcap;
-            const int64_t grow0 = (int64_t)g * kR;
-            // Q^T fragments (B operand): Q[j0 + lane/4][16 ks + 2 q4 ..] and 8 channels on.
-            uint32_t bq[NKS][2];
-            {
-                const bool okq = r8 < nr;
-                const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-                    a.Q + (okq ? ((grow0 + (int64_t)(j0 + r8) * R + r - 1) * H + h) * (2 * D) : 0));
+            // R, and draft token j' at plane r iff j' >= j - W + 1, else its depth-R row.
+            w.slide = pa.sliding && w.ring;
+            w.sbase = gc.T - s.W + 1 - gc.A;  // (T + j - W + 1) - A at j = 0
+            w.ndw = w.slide ? max(0, min(w.nw, w.sbase + w.j0 + w.nr - 1)) : 0;
+            w.nbr = w.slide ? max(0, w.j0 + w.nr - s.W) : 0;
+            w.slot0 = gc.A % s.Wcap;
+            w.fp = gc.fp;
+            w.fb = gc.fb;
+            // one Wcap-row box holds the window unless a fork position cuts deep rows
+            w.fast = pa.full_box && w.nw <= s.Wcap && s.Wcap + w.nblk + w.ndw + w.nbr <= KC &&
+                     (w.ring || !(gc.A < gc.fp && gc.A + s.Wcap > gc.fp));
+            w.koff = w.fast ? s.Wcap : w.nw;
+            w.nk = w.koff + w.nblk + w.ndw + w.nbr;
+            return w;
+        };
+        // The CTA's next unit whose group is valid (warp-uniform).
+        auto next_valid = [&](Unit& w) {
+            while (true) {
+                int u = 0;
+                if (lane == 0) u = atomicAdd(unit_next, 1);
+                u = __shfl_sync(0xffffffffu, u, 0);
+                if (u >= uend) return false;
+                w = describe(u);
+                if (w.ok) return true;
+            }
+        };
+        // Q^T fragments (B operand): Q[j0 + lane/4][16 ks + 2 q4 ..] and 8 channels on.
+        auto load_q = [&](const Unit& w, uint32_t (&b)[NKS][2]) {
+            const bool okq = r8 < w.nr;
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+                a.Q + (okq ? (((int64_t)w.g * kR + (int64_t)(w.j0 + r8) * R + w.r - 1) * H + w.h) * (2 * D) : 0));
 #pragma unroll
-                for (int ks = 0; ks < NKS; ++ks) {
-                    bq[ks][0] = okq ? __ldg(qp + 8 * ks + q4) : 0u;
-                    bq[ks][1] = okq ? __ldg(qp + 8 * ks + 4 + q4) : 0u;
+            for (int ks = 0; ks < NKS; ++ks) {
+                b[ks][0] = okq ? __ldg(qp + 8 * ks + q4) : 0u;
+                b[ks][1] = okq ? __ldg(qp + 8 * ks + 4 + q4) : 0u;
+            }
+        };
+        // Keys [k0, k0 + 16 nt) of unit w into the stage: 8-key groups of window keys
+        // contiguous in memory by TMA (lane 0), the rest (a group that wraps the ring,
+        // a partial group, draft tokens, plane-R keys of the sliding window, zero fill)
+        // by 16-byte copies.  The stage's earlier reads are done (caller's __syncwarp).
+        auto issue = [&](const Unit& w, int k0, uint8_t* stage, uint64_t* bar, bool qrows) {
+            const int nt = (min(KC, w.nk - k0) + 15) / 16;
+            const int64_t grow0 = (int64_t)w.g * kR;
+            // Rows of ring plane r (slot 0) and of the deep plane (position 0; deep_yp:
+            // the fork parent's) in the tensor maps' 2-D views.
+            const int64_t ring_y = ((((int64_t)a.layer * s.Bmax + w.seq) * H + w.h) * (R - 1) + (w.r - 1)) * s.Wcap;
+            const int64_t deep_y = (((int64_t)a.layer * s.Bmax + w.seq) * H + w.h) * s.Tmax;
+            const int64_t deep_yp = (((int64_t)a.layer * s.Bmax + w.fb) * H + w.h) * s.Tmax;
+            fence_proxy_async_smem();
+            // Source of key kk's 16-byte vector v, for the keys that go by copy.
+            auto key_src = [&](int kk, int v, const char*& ks_, const char*& vs_) -> bool {
+                int64_t off = v * 16;
+                if (kk < w.koff) {  // window key (position order: the chunked form)
+                    const int pos = w.A + kk;
+                    off += (w.ring ? ring_y + (w.slot0 + kk) % s.Wcap : (pos < w.fp ? deep_yp : deep_y) + pos) *
+                           (2 * D);
+                    ks_ = (w.ring ? s.kwin : s.kdeep) + off;
+                    vs_ = (w.ring ? s.vwin : s.vdeep) + off;
+                    return true;
+                }
+                int e = kk - w.koff;
+                if (e < w.nblk) {  // draft token e at plane r
+                    off += ((grow0 + (int64_t)e * R + w.r - 1) * H + w.h) * (2 * D);
+                    ks_ = a.Kb + off;
+                    vs_ = a.Vb + off;
+                    return true;
+                }
+                e -= w.nblk;
+                if (e < w.ndw) {  // sliding: window position at plane R
+                    const int pos = w.A + e;
+                    off += ((pos < w.fp ? deep_yp : deep_y) + pos) * (2 * D);
+                    ks_ = s.kdeep + off;
+                    vs_ = s.vdeep + off;
+                    return true;
+                }
+                e -= w.ndw;
+                if (e < w.nbr) {  // sliding: draft token e at plane R (its depth-R row)
+                    off += ((grow0 + (int64_t)e * R + R - 1) * H + w.h) * (2 * D);
+                    ks_ = a.Kb + off;
+                    vs_ = a.Vb + off;
+                    return true;
+                }
+                return false;  // past the unit's keys: zero fill
+            };
+            auto copy_key = [&](int kl, int v) {
+                const char* ks_ = a.Q;
+                const char* vs_ = a.Q;
+                const bool valid = key_src(k0 + kl, v, ks_, vs_);
+                const int c = v >> 2, v4 = v & 3;
+                uint8_t* dk = stage + c * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4);
+                if (!qrows || kl < KC - 8) cp_async16_zfill(dk, ks_, valid);  // else the row holds Q
+                cp_async16_zfill(dk + NCH * Lay::KCB, vs_, valid);
+            };
+            // The slice's query rows (zeros past nr) into key rows KC-8.. of the K part.
+            auto finish = [&]() {
+                if (qrows) {
+                    const int64_t grow0q = (int64_t)w.g * kR;
+                    for (int e = lane; e < 8 * VPR; e += 32) {
+                        const int i = e / VPR, v = e % VPR, kl = KC - 8 + i;
+                        const bool okq = i < w.nr;
+                        const char* qs = a.Q + (okq ? ((grow0q + (int64_t)(w.j0 + i) * R + w.r - 1) * H + w.h) *
+                                                              (2 * D) + v * 16
+                                                        : 0);
+                        const int c = v >> 2, v4 = v & 3;
+                        cp_async16_zfill(stage + c * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4), qs, okq);
+                    }
+                }
+                cp_async_mbar_arrive(bar);
+            };
+            if (w.fast) {
+                // The whole window in one box per column chunk (k0 = 0), then the
+                // chunk's other keys and zero fill by copies.
+                if (lane == 0) {
+                    mbar_expect_tx(bar, (uint32_t)(s.Wcap * 64 * NCH * 2));
+                    const int y = w.ring ? (int)ring_y : (int)((w.A < w.fp ? deep_yp : deep_y) + w.A);
+                    const CUtensorMap* mk = w.ring ? &tm.wkf : &tm.rkf;
+                    const CUtensorMap* mv = w.ring ? &tm.wvf : &tm.rvf;
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) {
+                        tma_load_2d(stage + c * Lay::KCB, mk, 32 * c, y, bar);
+                        tma_load_2d(stage + (NCH + c) * Lay::KCB, mv, 32 * c, y, bar);
+                    }
+                }
+                const int nrest = 16 * nt - s.Wcap;
+                for (int e = lane; e < nrest * VPR; e += 32) copy_key(s.Wcap + e / VPR, e % VPR);
+                finish();
+                return;
+            }
+            uint32_t tma_groups = 0;
+#pragma unroll
+            for (int gm = 0; gm < 2 * NT; ++gm) {
+                const int kk = k0 + 8 * gm;
+                if (gm < 2 * nt && kk + 8 <= w.nw) {
+                    // contiguous in one ring plane, or deep rows on one side of a fork position
+                    const bool contig = w.ring ? ((w.slot0 + kk) % s.Wcap) + 8 <= s.Wcap
+                                               : (w.A + kk < w.fp) == (w.A + kk + 7 < w.fp);
+                    if (contig) tma_groups |= 1u << gm;
                 }
             }
-            float o[NMT][4];
-#pragma unroll
-            for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-            float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-            // Global rows of the ring plane r (slot 0) / of the deep plane (position 0),
-            // in the tensor maps' 2-D views, and byte bases for the per-key copies.
-            const int64_t ring_y = ((((int64_t)a.layer * s.Bmax + gc.seq) * H + h) * (R - 1) + (r - 1)) * s.Wcap;
-            const int64_t deep_y = (((int64_t)a.layer * s.Bmax + gc.seq) * H + h) * s.Tmax;
-            for (int k0 = 0; k0 < nk; k0 += KC) {
-                const int kc = min(KC, nk - k0);
-                const int nt = (kc + 15) / 16;
-                // ---- load keys [k0, k0 + 16 nt) into the stage: 8-key groups of window
-                // keys contiguous in memory by TMA, the rest (a wrapping group, a
-                // partial group, block keys, zero fill) by 16-byte copies.
-                __syncwarp();
-                fence_proxy_async_smem();  // earlier reads of this stage come before new writes
-                uint32_t tma_groups = 0;   // bit m: group m of this chunk goes by TMA
-#pragma unroll
-                for (int gm = 0; gm < 2 * NT; ++gm) {
+            if (lane == 0) {
+                mbar_expect_tx(bar, (uint32_t)__popc(tma_groups) * 8 * 64 * NCH * 2);
+                uint32_t gmask = tma_groups;
+                while (gmask) {
+                    const int gm = __ffs(gmask) - 1;
+                    gmask &= gmask - 1;
                     const int kk = k0 + 8 * gm;
-                    if (gm < 2 * nt && kk + 8 <= nw) {
-                        const bool contig = !ring || ((slot0 + kk) % s.Wcap) + 8 <= s.Wcap;
-                        if (contig) tma_groups |= 1u << gm;
-                    }
-                }
-                if (lane == 0) {
-                    mbar_expect_tx(bar, (uint32_t)__popc(tma_groups) * 8 * 64 * NCH * 2);
-                    uint32_t gmask = tma_groups;
-                    while (gmask) {
-                        const int gm = __ffs(gmask) - 1;
-                        gmask &= gmask - 1;
-                        const int kk = k0 + 8 * gm;
-                        const int y = ring ? (int)(ring_y + (slot0 + kk) % s.Wcap) : (int)(deep_y + gc.A + kk);
-                        const CUtensorMap* mk = ring ? &tm.wk : &tm.rk;
-                        const CUtensorMap* mv = ring ? &tm.wv : &tm.rv;
+                    const int y = w.ring ? (int)(ring_y + (w.slot0 + kk) % s.Wcap)
+                                         : (int)((w.A + kk < w.fp ? deep_yp : deep_y) + w.A + kk);
+                    const CUtensorMap* mk = w.ring ? &tm.wk : &tm.rk;
+                    const CUtensorMap* mv = w.ring ? &tm.wv : &tm.rv;
 #pragma unroll
-                        for (int c = 0; c < NCH; ++c) {
-                            tma_load_2d(stage + c * Lay::KCB + gm * 512, mk, 32 * c, y, bar);
-                            tma_load_2d(stage + (NCH + c) * Lay::KCB + gm * 512, mv, 32 * c, y, bar);
-                        }
+                    for (int c = 0; c < NCH; ++c) {
+                        tma_load_2d(stage + c * Lay::KCB + gm * 512, mk, 32 * c, y, bar);
+                        tma_load_2d(stage + (NCH + c) * Lay::KCB + gm * 512, mv, 32 * c, y, bar);
                     }
                 }
-                // Per-key copies: (key, 16-byte vector) pairs of the other groups.
-                {
-                    constexpr int VPR = NCH * 4;  // 16-byte vectors per key row
-                    const uint32_t other = ((1u << (2 * nt)) - 1) & ~tma_groups;
-                    const int nother = __popc(other);
-                    for (int e = lane; e < nother * 8 * VPR; e += 32) {
-                        const int gi = e / (8 * VPR), rem = e % (8 * VPR);
-                        const int kr = rem / VPR, v = rem % VPR;
-                        // gi-th set bit of `other`
-                        uint32_t om = other;
-                        for (int z = 0; z < gi; ++z) om &= om - 1;
-                        const int gm = __ffs(om) - 1;
-                        const int kl = 8 * gm + kr;  // key within the chunk
-                        const int kk = k0 + kl;
-                        const char* ks_ = a.Q;
-                        const char* vs_ = a.Q;
-                        bool valid = true;
-                        if (kk < nw) {
-                            const int64_t row = ring ? ring_y + (slot0 + kk) % s.Wcap : deep_y + gc.A + kk;
-                            const int64_t off = row * (2 * D) + v * 16;
-                            ks_ = (ring ? s.kwin : s.kdeep) + off;
-                            vs_ = (ring ? s.vwin : s.vdeep) + off;
-                        } else if (kk < nw + nblk) {
-                            const int64_t off = ((grow0 + (int64_t)(kk - nw) * R + r - 1) * H + h) * (2 * D) + v * 16;
-                            ks_ = a.Kb + off;
-                            vs_ = a.Vb + off;
-                        } else if (kk < nw + nblk + ndw) {  // sliding: window position at plane R
-                            const int64_t off = (deep_y + gc.A + (kk - nw - nblk)) * (2 * D) + v * 16;
-                            ks_ = s.kdeep + off;
-                            vs_ = s.vdeep + off;
-                        } else if (kk < nk) {  // sliding: draft token at plane R (its depth-R row)
-                            const int64_t off =
-                                ((grow0 + (int64_t)(kk - nw - nblk - ndw) * R + R - 1) * H + h) * (2 * D) + v * 16;
-                            ks_ = a.Kb + off;
-                            vs_ = a.Vb + off;
-                        } else {
-                            valid = false;
-                        }
-                        const int c = v >> 2, v4 = v & 3;
-                        uint8_t* dk = stage + c * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4);
-                        cp_async16_zfill(dk, ks_, valid);
-                        cp_async16_zfill(dk + NCH * Lay::KCB, vs_, valid);
-                    }
-                    cp_async_mbar_arrive(bar);
-                }
-                if (!warp_wait(bar, phase & 1, abort_flag, s.err)) {
-                    wok = false;
-                    break;
-                }
-                ++phase;
-                const uint32_t sb = smem_ready(stage_a);
-                // ---- S^T = K Q^T for the chunk's 16-key tiles (independent chains)
-                float sc[NT][4];
+            }
+            uint32_t other = ((1u << (2 * nt)) - 1) & ~tma_groups;
+            while (other) {  // warp-uniform
+                const int gm = __ffs(other) - 1;
+                other &= other - 1;
+                for (int e = lane; e < 8 * VPR; e += 32) copy_key(8 * gm + e / VPR, e % VPR);
+            }
+            finish();
+        };
+
+        // The last arrival on a slice merges it: deep chunks in order, then the window
+        // partial, all read back from scratch.  Lane = (row lane/4, float4 column
+        // lane%4 + 4 v); the scale factors first (one round of loads), then the
+        // partials a few segments at a time.  Same arithmetic and order as the deep
+        // merge, so whoever merges writes the same bits.
+        auto resolve = [&](const Slice& w, int old) {
+            const bool last = __shfl_sync(0xffffffffu, old, 0) == w.E - 1;
+            if (!last) return;
+            if (lane == 0) *slice_counter(a, pa, w.g, w.j0, w.r, w.h) = 0;  // nothing else touches it
+            __syncwarp();  // lane 0's acquire, then every lane's reads
+            constexpr int NV = D / 16;
+            const int rr = lane >> 2, c4 = lane & 3;
+            const bool vr = rr < w.nr;
+            const int64_t ro = ((int64_t)w.g * kR + (int64_t)(w.j0 + rr) * R + w.r - 1) * H + w.h;
+            const int np = w.E - 1;  // segment np is the window
+            float2 ml[9];
+            float M = -INFINITY;
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt) {
-                    sc[tt][0] = sc[tt][1] = sc[tt][2] = sc[tt][3] = 0.f;
-                    if (tt < nt) {
+            for (int sg = 0; sg < 9; ++sg) {
+                ml[sg] = make_float2(-INFINITY, 0.f);
+                if (sg <= np && vr) ml[sg] = __ldcg(a.part_ml + ro * a.nseg + (sg < np ? sg : a.nsplit));
+                if (sg <= np) M = fmaxf(M, ml[sg].x);
+            }
+            float fs[9], L = 0.f;
+#pragma unroll
+            for (int sg = 0; sg < 9; ++sg) {
+                fs[sg] = ex2(ml[sg].x - M);
+                if (sg <= np) L = fmaf(ml[sg].y, fs[sg], L);
+            }
+            float4 acc[NV];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            constexpr int SB = NV >= 6 ? 1 : 2;  // segments per round of loads
+#pragma unroll
+            for (int sb = 0; sb < 9; sb += SB) {
+                if (sb > np) break;
+                float4 x[SB][NV];
+#pragma unroll
+                for (int i = 0; i < SB; ++i) {
+                    const int sg = sb + i;
+                    const float4* src = reinterpret_cast<const float4*>(
+                        a.part_o + (ro * a.nseg + (sg < np ? sg : a.nsplit)) * D);
+#pragma unroll
+                    for (int v = 0; v < NV; ++v)
+                        x[i][v] = (sg <= np && vr) ? __ldcg(src + c4 + 4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int i = 0; i < SB; ++i) {
+                    const int sg = sb + i;
+                    if (sg > np) break;
+                    const float f = fs[sg];
+#pragma unroll
+                    for (int v = 0; v < NV; ++v) {
+                        acc[v].x = fmaf(x[i][v].x, f, acc[v].x);
+                        acc[v].y = fmaf(x[i][v].y, f, acc[v].y);
+                        acc[v].z = fmaf(x[i][v].z, f, acc[v].z);
+                        acc[v].w = fmaf(x[i][v].w, f, acc[v].w);
+                    }
+                }
+            }
+            if (vr) {
+                const float inv = 1.f / L;
+                uint2* orow = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D);
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+                    orow[c4 + 4 * v] = make_uint2(pack_bf16(acc[v].x * inv, acc[v].y * inv),
+                                                  pack_bf16(acc[v].z * inv, acc[v].w * inv));
+                if (c4 == 0 && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
+            }
+        };
+
+        // One chunk of keys [k0, k0 + KC) of unit w from the stage at sb_in into the
+        // running (o, m, l) of rows ra, rb.
+        auto compute = [&](const Unit& w, int k0, uint32_t sb_in, const uint32_t (&bq)[NKS][2], float (&o)[NMT][4],
+                           float& m_a, float& m_b, float& l_a, float& l_b) {
+            const int nt = (min(KC, w.nk - k0) + 15) / 16;
+            const uint32_t sb = smem_ready(sb_in);
+            // Two 16-key tiles per pass of a loop that is not unrolled (the body is
+            // what every window warp runs, so it stays in the instruction cache),
+            // with the running maxima and sums rescaled once per pass.
+#pragma unroll 1
+            for (int t0 = 0; t0 < nt; t0 += 2) {
+                const bool two = t0 + 1 < nt;
+                // ---- S^T = K Q^T for the pass's tiles (independent chains)
+                float sc[2][4];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    sc[u][0] = sc[u][1] = sc[u][2] = sc[u][3] = 0.f;
+                    if (u == 0 || two) {
 #pragma unroll
                         for (int ks = 0; ks < NKS; ++ks) {
                             uint32_t a0, a1, a2, a3;
-                            ldsm_x4_r(sb + (ks >> 1) * Lay::KCB + (16 * tt + rk) * 64 + ((ks & 1) ? k_sw1 : k_sw0), a0,
-                                      a1, a2, a3);
-                            mma_16816(sc[tt], a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+                            ldsm_x4_r(sb + (ks >> 1) * Lay::KCB + (16 * (t0 + u) + rk) * 64 + ((ks & 1) ? k_sw1 : k_sw0),
+                                      a0, a1, a2, a3);
+                            mma_16816(sc[u], a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
                         }
                     }
                 }
-                // ---- visibility and the chunk's row maxima.  Key kk is visible to row j
-                // if it is a window key, or block token kk - nw <= j.
+                // ---- visibility and the pass's row maxima.  Key kk is visible to row j
+                // if it is a window key, or block token kk - koff <= j (sliding: per row).
                 float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt) {
-                    if (tt < nt) {
+                for (int u = 0; u < 2; ++u) {
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            const int kk = k0 + 16 * tt + r8 + 8 * hf;
-                            bool va, vb;
-                            if (!slide) {
-                                va = kk < nw || (kk < nk && kk - nw <= j0 + ra);
-                                vb = kk < nw || (kk < nk && kk - nw <= j0 + rb);
-                            } else {
-                                va = slide_visible(kk, j0 + ra, nw, nblk, ndw, nk, sbase, s.W);
-                                vb = slide_visible(kk, j0 + rb, nw, nblk, ndw, nk, sbase, s.W);
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int kk = k0 + 16 * (t0 + u) + r8 + 8 * hf;
+                        bool va, vb;
+                        if (u == 1 && !two) {
+                            va = vb = false;
+                        } else if (kk < w.koff) {
+                            // window key: offset i from A (whole-window ring: slot kk)
+                            int i = kk;
+                            if (w.fast && w.ring) {
+                                i = kk + s.Wcap - w.slot0;
+                                if (i >= s.Wcap) i -= s.Wcap;
                             }
-                            float& xa = sc[tt][2 * hf];
-                            float& xb = sc[tt][2 * hf + 1];
-                            xa = va ? xa * c2 : -INFINITY;
-                            xb = vb ? xb * c2 : -INFINITY;
-                            mx_a = fmaxf(mx_a, xa);
-                            mx_b = fmaxf(mx_b, xb);
+                            va = vb = i < w.nw;
+                            if (w.slide) {
+                                va = va && i >= w.sbase + w.j0 + ra;
+                                vb = vb && i >= w.sbase + w.j0 + rb;
+                            }
+                        } else if (!w.slide) {
+                            const int e = kk - w.koff;
+                            va = e < w.nblk && e <= w.j0 + ra;
+                            vb = e < w.nblk && e <= w.j0 + rb;
+                        } else {
+                            const int e = kk - w.koff;
+                            va = slide_visible(e, w.j0 + ra, w.nblk, w.ndw, w.nbr, w.sbase, s.W);
+                            vb = slide_visible(e, w.j0 + rb, w.nblk, w.ndw, w.nbr, w.sbase, s.W);
                         }
+                        float& xa = sc[u][2 * hf];
+                        float& xb = sc[u][2 * hf + 1];
+                        xa = va ? xa * c2 : -INFINITY;
+                        xb = vb ? xb * c2 : -INFINITY;
+                        mx_a = fmaxf(mx_a, xa);
+                        mx_b = fmaxf(mx_b, xb);
                     }
                 }
 #pragma unroll
@@ -885,55 +1108,46 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     o[mt][1] *= al_b;
                     o[mt][3] *= al_b;
                 }
-                // ---- probabilities and P^T fragments (8x8 transposes of the S^T fragments)
-                uint32_t pb[NT][2];
+                // ---- probabilities, P^T fragments (8x8 transposes of the S^T fragments)
+                // and O^T += V^T P^T
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt) {
-                    if (tt < nt) {
-                        const float p0 = mn_a == -INFINITY ? 0.f : ex2(sc[tt][0] - mn_a);
-                        const float p1 = mn_b == -INFINITY ? 0.f : ex2(sc[tt][1] - mn_b);
-                        const float p2 = mn_a == -INFINITY ? 0.f : ex2(sc[tt][2] - mn_a);
-                        const float p3 = mn_b == -INFINITY ? 0.f : ex2(sc[tt][3] - mn_b);
+                for (int u = 0; u < 2; ++u) {
+                    if (u == 0 || two) {
+                        const float p0 = mn_a == -INFINITY ? 0.f : ex2(sc[u][0] - mn_a);
+                        const float p1 = mn_b == -INFINITY ? 0.f : ex2(sc[u][1] - mn_b);
+                        const float p2 = mn_a == -INFINITY ? 0.f : ex2(sc[u][2] - mn_a);
+                        const float p3 = mn_b == -INFINITY ? 0.f : ex2(sc[u][3] - mn_b);
                         l_a += p0 + p2;
                         l_b += p1 + p3;
-                        pb[tt][0] = movmatrix_t(pack_bf16(p0, p1));
-                        pb[tt][1] = movmatrix_t(pack_bf16(p2, p3));
-                    } else {
-                        pb[tt][0] = pb[tt][1] = 0u;
-                    }
-                }
-                // ---- O^T += V^T P^T (one chain per 16-channel tile)
+                        const uint32_t pb0 = movmatrix_t(pack_bf16(p0, p1));
+                        const uint32_t pb1 = movmatrix_t(pack_bf16(p2, p3));
 #pragma unroll
-                for (int mt = 0; mt < NMT; ++mt) {
-#pragma unroll
-                    for (int tt = 0; tt < NT; ++tt) {
-                        if (tt < nt) {
+                        for (int mt = 0; mt < NMT; ++mt) {
                             uint32_t a0, a1, a2, a3;
-                            ldsm_x4_t_r(sb + NCH * Lay::KCB + (mt >> 1) * Lay::KCB + (16 * tt + rv) * 64 +
+                            ldsm_x4_t_r(sb + NCH * Lay::KCB + (mt >> 1) * Lay::KCB + (16 * (t0 + u) + rv) * 64 +
                                             ((mt & 1) ? v_sw1 : v_sw0),
                                         a0, a1, a2, a3);
-                            mma_16816(o[mt], a0, a1, a2, a3, pb[tt][0], pb[tt][1]);
+                            mma_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
                         }
                     }
                 }
             }
-            if (!wok) break;
-            // ---- the unit's end: row sums across the lanes of a row
+            __syncwarp();  // every lane is done reading the stage
+        };
+
+        // Publish a unit's partial (segment nsplit of its rows) and arrive on its
+        // slice; returns lane 0's counter value before the arrival.
+        auto publish = [&](const Slice& w, const float (&o)[NMT][4], float m_a, float m_b, float l_a, float l_b) {
 #pragma unroll
             for (int o2 = 4; o2 < 32; o2 <<= 1) {
                 l_a += __shfl_xor_sync(0xffffffffu, l_a, o2);
                 l_b += __shfl_xor_sync(0xffffffffu, l_b, o2);
             }
-            int32_t* cp = slice_counter(a, pa, g, j0, r, h);
-            bool last = false;
-            if (lane == 0) last = ld_acquire(cp) == gc.E - 1;
-            last = __shfl_sync(0xffffffffu, last, 0);
-            const bool va = ra < nr, vb = rb < nr;
-            const int64_t ro_a = (grow0 + (int64_t)(j0 + ra) * R + r - 1) * H + h;
-            const int64_t ro_b = (grow0 + (int64_t)(j0 + rb) * R + r - 1) * H + h;
-            if (!last) {
-                // Publish this unit's partial (segment nsplit), then arrive.
-                const int64_t pa_ = ro_a * a.nseg + a.nsplit, pb_ = ro_b * a.nseg + a.nsplit;
+            {
+                const bool va = ra < w.nr, vb = rb < w.nr;
+                const int64_t grow0 = (int64_t)w.g * kR;
+                const int64_t pa_ = ((grow0 + (int64_t)(w.j0 + ra) * R + w.r - 1) * H + w.h) * a.nseg + a.nsplit;
+                const int64_t pb_ = ((grow0 + (int64_t)(w.j0 + rb) * R + w.r - 1) * H + w.h) * a.nseg + a.nsplit;
 #pragma unroll
                 for (int mt = 0; mt < NMT; ++mt) {
                     const int ch = 16 * mt + r8;
@@ -950,103 +1164,220 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     if (va) a.part_ml[pa_] = make_float2(m_a, l_a);
                     if (vb) a.part_ml[pb_] = make_float2(m_b, l_b);
                 }
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) last = atomicAdd(cp, 1) == gc.E - 1;
-                last = __shfl_sync(0xffffffffu, last, 0);
             }
-            if (!last) continue;
-            if (lane == 0) *cp = 0;
-            __threadfence();
-            // ---- merge rows ra, rb of this lane's channels with the deep chunks'
-            // partials, segments in the fixed order (deep chunks, then this window).
-            const int np = gc.E - 1;
-            float Ma = m_a, Mb = m_b;
-            for (int sg = 0; sg < np; ++sg) {
-                if (va) Ma = fmaxf(Ma, __ldcg(a.part_ml + ro_a * a.nseg + sg).x);
-                if (vb) Mb = fmaxf(Mb, __ldcg(a.part_ml + ro_b * a.nseg + sg).x);
-            }
-            float acc[NMT][4];
-#pragma unroll
-            for (int mt = 0; mt < NMT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-            float La = 0.f, Lb = 0.f;
-            for (int sg = 0; sg < np; ++sg) {
-                if (va) {
-                    const float2 ml = __ldcg(a.part_ml + ro_a * a.nseg + sg);
-                    const float f = ex2(ml.x - Ma);
-                    La = fmaf(ml.y, f, La);
-                    const float* po = a.part_o + (ro_a * a.nseg + sg) * D + r8;
-#pragma unroll
-                    for (int mt = 0; mt < NMT; ++mt) {
-                        acc[mt][0] = fmaf(__ldcg(po + 16 * mt), f, acc[mt][0]);
-                        acc[mt][2] = fmaf(__ldcg(po + 16 * mt + 8), f, acc[mt][2]);
+            __syncwarp();  // orders every lane's partial writes before lane 0's release
+            return lane == 0 ? arrive_acq_rel(slice_counter(a, pa, w.g, w.j0, w.r, w.h)) : 0;
+        };
+
+        if constexpr (RING) {
+            // ---- stage ring: full[st] (33 arrivals: 32 lanes' copies + the expect_tx),
+            // empty[st] (the consumer that read it), the unit in desc[st].
+            static_assert(sizeof(Unit) <= Lay::DESC_BYTES, "unit descriptor");
+            const int NS = deep_cta ? NWW : Lay::NW_FULL;
+            uint8_t* sring = sm + (deep_cta ? Lay::OFF_W : 0);
+            uint64_t* full = wbar;
+            uint64_t* empty = wbar + Lay::NWARPS;
+            Unit* desc = reinterpret_cast<Unit*>(sm + Lay::OFF_DESC);
+            int* ticket = reinterpret_cast<int*>(sm + Lay::OFF_MISC + 20);
+            // A consumer waits for its ticket to be issued into its stage before it
+            // looks at the stage's barrier: a ticket a full ring ahead would otherwise
+            // see the parity of the stage's previous use and pass at once.  (Shared
+            // memory is one coherent store for the CTA: once the ticket shows, the
+            // barrier's earlier phases show too.)
+            volatile int* issued = reinterpret_cast<volatile int*>(sm + Lay::OFF_ISS);
+            // Two producer warps (even and odd tickets) where the CTA has the warps.
+            const int NP = (deep_cta ? Lay::NWARPS - kDeepWarps : Lay::NWARPS) >= 4 ? 2 : 1;
+            const int ub = (int)(ub64 < pa.nunits ? ub64 : pa.nunits);
+            const int ntk = uend > ub ? uend - ub : 0;
+            if (warp >= wfirst && warp < wfirst + NP) {
+                // ---------------------------------------- producers
+                for (int idx = warp - wfirst; idx < ntk; idx += NP) {
+                    const int st = idx % NS;
+                    if (idx >= NS && !warp_wait(empty + st, ((idx / NS) - 1) & 1, abort_flag, s.err)) break;
+                    Unit w = describe(ub + idx);
+                    // every unit here is one chunk with room for its queries
+                    if (w.ok && w.nk > KC - 8) {
+                        if (lane == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
+                        w.ok = false;
                     }
-                }
-                if (vb) {
-                    const float2 ml = __ldcg(a.part_ml + ro_b * a.nseg + sg);
-                    const float f = ex2(ml.x - Mb);
-                    Lb = fmaf(ml.y, f, Lb);
-                    const float* po = a.part_o + (ro_b * a.nseg + sg) * D + r8;
-#pragma unroll
-                    for (int mt = 0; mt < NMT; ++mt) {
-                        acc[mt][1] = fmaf(__ldcg(po + 16 * mt), f, acc[mt][1]);
-                        acc[mt][3] = fmaf(__ldcg(po + 16 * mt + 8), f, acc[mt][3]);
+                    if (lane == 0) desc[st] = w;  // published by lane 0's arrival below
+                    if (w.ok) {
+                        issue(w, 0, sring + st * Lay::WSTAGE, full + st, true);
+                    } else {
+                        if (lane == 0) mbar_arrive(full + st);
+                        cp_async_mbar_arrive(full + st);
                     }
+                    if (lane == 0) issued[st] = idx;
                 }
-            }
-            const float fa = ex2(m_a - Ma), fb = ex2(m_b - Mb);
-            La = fmaf(l_a, fa, La);
-            Lb = fmaf(l_b, fb, Lb);
+                // This warp's copies land before it leaves (the tensor copies of a ring
+                // that gave up are waited for at the end of the kernel).
+                cp_async_wait_all();
+            } else {
+                // ---------------------------------------- consumers
+                Slice pw;  // the slice whose arrival is looked at next
+                int pold = 0;
+                bool pend = false;
+                while (true) {
+                    int t = 0;
+                    if (lane == 0) t = atomicAdd(ticket, 1);
+                    t = __shfl_sync(0xffffffffu, t, 0);
+                    const bool have = t < ntk;
+                    int old_now = 0;
+                    bool mine = false;
+                    Slice cs{};
+                    if (have) {
+                        const int st = t % NS;
+                        int okc = 1;
+                        if (lane == 0) okc = count_wait(issued + st, t - 1, abort_flag, s.err);
+                        if (!__shfl_sync(0xffffffffu, okc, 0)) break;
+                        if (!warp_wait(full + st, (t / NS) & 1, abort_flag, s.err)) break;
+                        const Unit w = desc[st];
+                        const uint32_t sa = smem_u32(sring + st * Lay::WSTAGE);
+                        float o[NMT][4];
+                        float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+                        if (w.ok) {
+                            // Q^T fragments from the stage's last 8 key rows of each column chunk
+                            uint32_t bq[NKS][2];
+                            const int qr = KC - 8 + (lane & 7);
 #pragma unroll
-            for (int mt = 0; mt < NMT; ++mt) {
-                o[mt][0] = fmaf(o[mt][0], fa, acc[mt][0]);
-                o[mt][2] = fmaf(o[mt][2], fa, acc[mt][2]);
-                o[mt][1] = fmaf(o[mt][1], fb, acc[mt][1]);
-                o[mt][3] = fmaf(o[mt][3], fb, acc[mt][3]);
-            }
-            const float ia = 1.f / La, ib = 1.f / Lb;
-            __nv_bfloat16* Oa = reinterpret_cast<__nv_bfloat16*>(a.O) + ro_a * D + r8;
-            __nv_bfloat16* Ob = reinterpret_cast<__nv_bfloat16*>(a.O) + ro_b * D + r8;
+                            for (int c = 0; c < NCH; ++c)
+                                ldsm_x4_r(smem_ready(sa) + c * Lay::KCB + qr * 64 + (((lane >> 3) ^ ((qr >> 1) & 3)) << 4),
+                                          bq[2 * c][0], bq[2 * c][1], bq[2 * c + 1][0], bq[2 * c + 1][1]);
 #pragma unroll
-            for (int mt = 0; mt < NMT; ++mt) {
-                if (va) {
-                    Oa[16 * mt] = __float2bfloat16_rn(o[mt][0] * ia);
-                    Oa[16 * mt + 8] = __float2bfloat16_rn(o[mt][2] * ia);
-                }
-                if (vb) {
-                    Ob[16 * mt] = __float2bfloat16_rn(o[mt][1] * ib);
-                    Ob[16 * mt + 8] = __float2bfloat16_rn(o[mt][3] * ib);
+                            for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+                            compute(w, 0, sa, bq, o, m_a, m_b, l_a, l_b);
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(empty + st);  // the stage is free again
+                        if (w.ok) {
+                            cs = Slice{w.g, w.h, w.r, w.j0, w.nr, w.E};
+                            old_now = publish(cs, o, m_a, m_b, l_a, l_b);
+                            mine = true;
+                        }
+                    }
+                    // The older arrival has returned by now: merge its slice if it was the
+                    // last; after the last ticket, the final arrival too.
+#pragma unroll 1
+                    for (int pass = 0; pass < 2; ++pass) {
+                        if (pend) resolve(pw, pold);
+                        pend = false;
+                        if (mine && pass == 0) {
+                            pw = cs;
+                            pold = old_now;
+                            pend = true;
+                        }
+                        if (have || !pend) break;
+                    }
+                    if (!have) break;
                 }
             }
-            if (r8 == 0 && a.lse) {
-                if (va) a.lse[ro_a] = (Ma + log2f(La)) * 0.69314718055994531f;
-                if (vb) a.lse[ro_b] = (Mb + log2f(Lb)) * 0.69314718055994531f;
+        } else {
+            uint32_t phase = 0;
+            bool wok = true;
+            // One site per step (next unit, issue, publish, merge) keeps the loop's code
+            // small.  Each pass: pick the next load (the current unit's next chunk, or a
+            // new unit), issue it, publish and arrive for a unit that just ended, merge
+            // the slice of the arrival before it if that was the last, then wait for
+            // the load and compute on it.
+            Unit cur{};
+            int k0 = 0;
+            bool started = false;
+            Slice pw;  // the slice whose arrival is looked at next
+            int pold = 0;
+            bool pend = false;
+            uint32_t bq[NKS][2];
+            float o[NMT][4];
+            float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+            while (true) {
+                const Slice cs{cur.g, cur.h, cur.r, cur.j0, cur.nr, cur.E};
+                Unit nxt;
+                int nk0 = 0;
+                bool have;
+                if (started && k0 + KC < cur.nk) {
+                    nxt = cur;
+                    nk0 = k0 + KC;
+                    have = true;
+                } else {
+                    have = next_valid(nxt);
+                }
+                const bool ended = started && nk0 == 0;
+                if (have) {
+                    issue(nxt, nk0, stage, bar, false);
+                    if (nk0 == 0) load_q(nxt, bq);  // the current unit's compute is done with bq
+                }
+                int old_now = 0;
+                if (ended) {
+                    const Slice& w = cs;
+                    // ---- publish the unit's partial (segment nsplit) and arrive; whether it
+                    // was the last arrival is looked at when the next unit ends.
+                    old_now = publish(w, o, m_a, m_b, l_a, l_b);
+                }
+                // The older arrival has returned by now: if it was its slice's last, merge
+                // the slice while the next keys are in flight.  After the last unit, the
+                // final arrival is looked at too.
+#pragma unroll 1
+                for (int pass = 0; pass < 2; ++pass) {
+                    if (pend) resolve(pw, pold);
+                    pend = false;
+                    if (ended && pass == 0) {
+                        pw = cs;
+                        pold = old_now;
+                        pend = true;
+                    }
+                    if (have || !pend) break;
+                }
+                if (!have) break;
+                cur = nxt;
+                k0 = nk0;
+                started = true;
+                if (k0 == 0) {
+#pragma unroll
+                    for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+                    m_a = m_b = -INFINITY;
+                    l_a = l_b = 0.f;
+                }
+                if (!warp_wait(bar, phase & 1, abort_flag, s.err)) {
+                    wok = false;
+                    break;
+                }
+                ++phase;
+                compute(cur, k0, stage_a, bq, o, m_a, m_b, l_a, l_b);
             }
-        }
-        if (!wok) {
-            // Let this warp's copies land before the CTA's shared memory goes away.
-            volatile int no_abort = 0;
-            cp_async_wait_all();
-            mbar_wait(bar, phase & 1, &no_abort, s.err);
+            if (!wok) {
+                // Let this warp's copies land before the CTA's shared memory goes away.
+                volatile int no_abort = 0;
+                cp_async_wait_all();
+                mbar_wait(bar, phase & 1, &no_abort, s.err);
+            }
         }
     }
+
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (RING && threadIdx.x == 0 && *abort_flag) {
+        // A ring that gave up may still have tensor copies in flight: wait for the
+        // last phase issued into each stage before the shared memory goes away.
+        const int NS = deep_cta ? NWW : Lay::NW_FULL;
+        const int* iss = reinterpret_cast<const int*>(sm + Lay::OFF_ISS);
+        volatile int no_abort = 0;
+        for (int st = 0; st < NS; ++st)
+            if (iss[st] >= 0) mbar_wait(wbar + st, (iss[st] / NS) & 1, &no_abort, s.err);
+    }
     if (deep_cta && warp == 5) tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
-template <int D, int MT, int ST, int NWW, int KC>
+template <int D, int MT, int ST, int NWW, int KC, bool RING>
 cudaError_t launch_p(const PMaps& tm, const VerifyArgs& a, const PArgs& pa, int grid, cudaStream_t st) {
     using Lay = PLayout<D, MT, ST, NWW, KC>;
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
     static PerDeviceOnce configured;
     cudaError_t ce = per_device_once(configured, [] {
-        cudaError_t e = cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC>,
+        cudaError_t e = cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC, RING>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
         if (e != cudaSuccess) return e;
-        return cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC>,
+        return cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC, RING>,
                                     cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     });
     if (ce != cudaSuccess) return ce;
@@ -1060,12 +1391,22 @@ cudaError_t launch_p(const PMaps& tm, const VerifyArgs& a, const PArgs& pa, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, persist_kernel<D, MT, ST, NWW, KC>, tm, a, pa);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, persist_kernel<D, MT, ST, NWW, KC, RING>, tm, a, pa);
     ripe_count_launch();
     return e;
 }
 
 }  // namespace
+
+// Keys per window chunk of the instantiation for (d, mt).
+static int persist_kc(int d, int mt) { return d == 128 && mt == 2 ? 48 : 80; }
+
+// Whether the window units run through the stage ring: every unit one chunk (the
+// whole window, the draft tokens) with 8 key rows left for its queries, no sliding
+// window (whose units read more keys).
+bool persist_ring_ok(int d, int mt, int Wcap, int k, int sliding, int full_box) {
+    return !sliding && full_box && Wcap + k <= persist_kc(d, mt) - 8;
+}
 
 // Window warps a CTA of each role runs, for the planner's cost model.
 void persist_shape(int d, int mt, int* nww_deep, int* nww_other) {
@@ -1087,9 +1428,10 @@ void persist_shape(int d, int mt, int* nww_deep, int* nww_other) {
 
 cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int32_t* cnt, int pd, int n_lo, int n_hi,
                            int ndeep, int nunits, int grid, int mt, long long probe_cycles, int sliding,
-                           cudaStream_t st) {
+                           int full_box, cudaStream_t st) {
     // Cache maps: 0 deep K, 1 deep V (64-row boxes); 6 ring K, 7 ring V, 8 deep K,
-    // 9 deep V (8-row boxes); plus one of this call's Q.
+    // 9 deep V (8-row boxes); 10-13 the same four in Wcap-row boxes; plus one of
+    // this call's Q.
     PMaps tm;
     const CUtensorMap* cm = reinterpret_cast<const CUtensorMap*>(tmaps);
     tm.dk = cm[0];
@@ -1098,18 +1440,26 @@ cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int32_t* c
     tm.wv = cm[7];
     tm.rk = cm[8];
     tm.rv = cm[9];
+    tm.wkf = cm[10];
+    tm.wvf = cm[11];
+    tm.rkf = cm[12];
+    tm.rvf = cm[13];
     VerifyArgs a = args;
     if (!make_q_map(&tm.q, a)) return cudaErrorInvalidValue;
-    PArgs pa{cnt, pd, n_lo, n_hi, ndeep, nunits, probe_cycles, sliding};
+    PArgs pa{cnt, pd, n_lo, n_hi, ndeep, nunits, probe_cycles, sliding, full_box};
     const int d = a.s.d;
-    if (mt == 1) {
-        if (d == 64) return launch_p<64, 1, 4, 6, 80>(tm, a, pa, grid, st);
-        if (d == 96) return launch_p<96, 1, 4, 4, 80>(tm, a, pa, grid, st);
-        if (d == 128) return launch_p<128, 1, 3, 3, 80>(tm, a, pa, grid, st);
-    } else {
-        if (d == 64) return launch_p<64, 2, 4, 5, 80>(tm, a, pa, grid, st);
-        if (d == 96) return launch_p<96, 2, 3, 3, 80>(tm, a, pa, grid, st);
-        if (d == 128) return launch_p<128, 2, 3, 2, 48>(tm, a, pa, grid, st);
-    }
+    // The stage ring when every unit is one chunk with room for its queries.
+    const bool ring = persist_ring_ok(d, mt, a.s.Wcap, a.ba.k, sliding, full_box);
+#define RIPE_LAUNCH(D_, MT_, ST_, NWW_, KC_)                                              \
+    if (d == D_ && mt == MT_)                                                          \
+        return ring ? launch_p<D_, MT_, ST_, NWW_, KC_, true>(tm, a, pa, grid, st)      \
+                    : launch_p<D_, MT_, ST_, NWW_, KC_, false>(tm, a, pa, grid, st);
+    RIPE_LAUNCH(64, 1, 4, 6, 80)
+    RIPE_LAUNCH(96, 1, 4, 4, 80)
+    RIPE_LAUNCH(128, 1, 3, 3, 80)
+    RIPE_LAUNCH(64, 2, 4, 5, 80)
+    RIPE_LAUNCH(96, 2, 3, 3, 80)
+    RIPE_LAUNCH(128, 2, 3, 2, 48)
+#undef RIPE_LAUNCH
     return cudaErrorInvalidValue;
 }

@@ -86,6 +86,72 @@ __global__ void reset_kernel(StoreView s, const int32_t* __restrict__ seq_ids, i
     s.len[b] = 0;
     s.ws[b] = 0;
     s.rfloor[b] = 0;
+    s.fbase[b] = b;  // a released fork no longer reads its parent
+    s.fpos[b] = 0;
+}
+
+// Every sequence starts as its own deep-plane owner (not a fork).
+__global__ void init_meta_kernel(StoreView s) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < s.Bmax) s.fbase[b] = b;
+}
+
+// A (parent, child) pair of ripe_fork is valid when both ids are in range and
+// distinct and the parent is not itself a fork.
+__device__ __forceinline__ bool fork_pair_ok(const StoreView& s, int p, int c) {
+    return p >= 0 && p < s.Bmax && c >= 0 && c < s.Bmax && p != c && s.fbase[p] == p;
+}
+
+// Branch fork (LoopSpec article, deployment section: a KV cache per branch): the
+// child takes copies of the parent's deep rows from its fork position
+// f = floor64(T) to T and of the parent's whole ring; rows below f stay in the
+// parent and are read through fbase/fpos.  16-byte vectors; per pair and (layer,
+// head) 64 deep rows (those at f + i < T) and (R-1)*Wcap ring rows.
+__global__ void fork_copy_kernel(StoreView s, const int32_t* __restrict__ parents,
+                                 const int32_t* __restrict__ children, int nseq) {
+    const int vecs = s.d * s.esize / 16;
+    const int ring_rows = (s.R - 1) * s.Wcap;
+    const int rows = 64 + ring_rows;
+    const int64_t total = (int64_t)nseq * s.L * s.H * rows * vecs;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        int64_t x = e;
+        const int v = (int)(x % vecs); x /= vecs;
+        const int row = (int)(x % rows); x /= rows;
+        const int h = (int)(x % s.H); x /= s.H;
+        const int l = (int)(x % s.L);
+        const int i = (int)(x / s.L);
+        const int p = parents[i], c = children[i];
+        if (!fork_pair_ok(s, p, c)) continue;
+        if (row < 64) {
+            const int T = s.len[p];
+            const int64_t pos = (int64_t)(T / 64 * 64) + row;
+            if (pos >= T) continue;
+            const int64_t src = deep_row(s, l, p, h, pos) + v * 16, dst = deep_row(s, l, c, h, pos) + v * 16;
+            *reinterpret_cast<uint4*>(s.kdeep + dst) = *reinterpret_cast<const uint4*>(s.kdeep + src);
+            *reinterpret_cast<uint4*>(s.vdeep + dst) = *reinterpret_cast<const uint4*>(s.vdeep + src);
+        } else {
+            const int rr = row - 64;
+            const int r = rr / s.Wcap + 1, slot = rr % s.Wcap;
+            const int64_t src = ring_row(s, l, p, h, r, slot) + v * 16, dst = ring_row(s, l, c, h, r, slot) + v * 16;
+            *reinterpret_cast<uint4*>(s.kwin + dst) = *reinterpret_cast<const uint4*>(s.kwin + src);
+            *reinterpret_cast<uint4*>(s.vwin + dst) = *reinterpret_cast<const uint4*>(s.vwin + src);
+        }
+    }
+}
+
+__global__ void fork_meta_kernel(StoreView s, const int32_t* __restrict__ parents,
+                                 const int32_t* __restrict__ children, int nseq) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nseq) return;
+    const int p = parents[i], c = children[i];
+    if (!fork_pair_ok(s, p, c)) { set_device_error(s.err, RIPE_DEVERR_FORK); return; }
+    const int T = s.len[p];
+    s.len[c] = T;
+    s.ws[c] = s.ws[p];
+    s.rfloor[c] = s.rfloor[p];
+    s.fbase[c] = p;
+    s.fpos[c] = T / 64 * 64;
 }
 
 // Rollback to the confirmed prefix (LoopSpec article, section on the second
@@ -101,7 +167,8 @@ __global__ void truncate_kernel(StoreView s, const int32_t* __restrict__ seq_ids
     if (b < 0 || b >= s.Bmax) { set_device_error(s.err, RIPE_DEVERR_SEQ_RANGE); return; }
     int T = s.len[b];
     const int t = new_len[i];
-    if (t < 0) { set_device_error(s.err, RIPE_DEVERR_COUNT); return; }
+    // A fork is never cut below its fork position (release it instead).
+    if (t < 0 || (s.fbase[b] != b && t < s.fpos[b])) { set_device_error(s.err, RIPE_DEVERR_COUNT); return; }
     if (t < T) T = t;
     const int rf = min(s.rfloor[b], T);
     s.len[b] = T;
@@ -158,6 +225,8 @@ __global__ void set_meta_kernel(StoreView s, int b, int T) {
     s.len[b] = T;
     s.ws[b] = T - s.Wcap > 0 ? T - s.Wcap : 0;
     s.rfloor[b] = s.ws[b];
+    s.fbase[b] = b;
+    s.fpos[b] = 0;
 }
 
 }  // namespace
@@ -182,6 +251,22 @@ cudaError_t launch_evict(const ripe_cache_s* c, const int32_t* seq_ids, int nseq
 cudaError_t launch_reset(const ripe_cache_s* c, const int32_t* seq_ids, int nseq, cudaStream_t st) {
     reset_kernel<<<(nseq + 127) / 128, 128, 0, st>>>(store_view(c), seq_ids, nseq);
     ripe_count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_init_meta(const ripe_cache_s* c, cudaStream_t st) {
+    init_meta_kernel<<<(c->Bmax + 127) / 128, 128, 0, st>>>(store_view(c));
+    ripe_count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fork(const ripe_cache_s* c, const int32_t* parents, const int32_t* children, int nseq,
+                        cudaStream_t st) {
+    StoreView s = store_view(c);
+    const int64_t total = (int64_t)nseq * s.L * s.H * (64 + (s.R - 1) * s.Wcap) * (s.d * s.esize / 16);
+    fork_copy_kernel<<<grid_for(total, kThreads), kThreads, 0, st>>>(s, parents, children, nseq);
+    fork_meta_kernel<<<(nseq + 127) / 128, 128, 0, st>>>(s, parents, children, nseq);
+    ripe_count_launch(2);
     return cudaGetLastError();
 }
 

@@ -142,7 +142,10 @@ seg_kernel(VerifyArgs a, int seg_first, int seg_count, int KT, int ST) {
                 off = ring_row(s, a.layer, b, h, r, slot);
                 kb = s.kwin; vb = s.vwin;
             } else {
-                off = deep_row(s, a.layer, b, h, p);
+                // a fork reads its parent's deep plane below its fork position
+                const int fp = s.fpos[b];
+                if (p < fp) n = min(n, fp - p);
+                off = deep_row(s, a.layer, deep_owner(s, b, p), h, p);
                 kb = s.kdeep; vb = s.vdeep;
             }
             bulk_load(dk + (size_t)(key - k0) * rowb, kb + off, (uint32_t)(n * rowb), full + st);
@@ -560,7 +563,7 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
         // The test hook is consumed by the launch it applies to.
         const long long probe = const_cast<ripe_cache_s*>(c)->probe_cycles.exchange(0);
         e = launch_persist(c->tmaps, a, reinterpret_cast<int32_t*>(cnt), plan.pd, plan.n_lo, plan.n_hi, plan.ndeep,
-                           plan.nunits, plan.grid, plan.mt, probe, ba.sliding, st);
+                           plan.nunits, plan.grid, plan.mt, probe, ba.sliding, c->full_box ? 1 : 0, st);
         if (e != cudaSuccess) return e;
     } else if (plan.fused) {
         // The whole call in one kernel; programmatic dependent launch lets its

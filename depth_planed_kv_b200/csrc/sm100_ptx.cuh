@@ -66,6 +66,26 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     }
 }
 
+// Wait until *count (raised by another warp of the CTA) is above v, bounded and
+// abortable like mbar_wait_slow.
+static __device__ __noinline__ bool count_wait_slow(volatile int* count, int v, volatile int* abort, int32_t* err,
+                                                    long long limit = (1ll << 31)) {
+    const long long t0 = clock64();
+    while (true) {
+        if (*count > v) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+            *abort = 1;
+            set_device_error(err, RIPE_DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool count_wait(volatile int* count, int v, volatile int* abort, int32_t* err) {
+    if (*count > v) return true;
+    return count_wait_slow(count, v, abort, err);
+}
+
 // Wait for the phase of `parity` to complete.  Gives up after ~2^31 clock
 // cycles (about a second), or as soon as another role has set *abort; on
 // give-up it records RIPE_DEVERR_TIMEOUT and returns false.

@@ -36,7 +36,8 @@ RIPE_ERR_UNSUPPORTED = 7
 RIPE_ERR_CAPTURING = 8
 RIPE_BF16 = 0
 RIPE_F32 = 1
-DEVERR_NAMES = {0: "none", 1: "seq_range", 2: "capacity", 3: "count", 4: "ctx", 5: "branch"}
+DEVERR_NAMES = {0: "none", 1: "seq_range", 2: "capacity", 3: "count", 4: "ctx", 5: "branch", 6: "timeout",
+                7: "fork"}
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -62,6 +63,8 @@ _sig("ripe_cache_reset", [_P, _P, _I, _P])
 _sig("ripe_append", [_P, _P, _P, _I, _P, _P, _I, _P])
 _sig("ripe_evict", [_P, _P, _I, _P])
 _sig("ripe_truncate", [_P, _P, _P, _I, _P])
+_sig("ripe_fork", [_P, _P, _P, _I, _P])
+_sig("ripe_read_forks", [_P, _P, _P, _P])
 _sig("ripe_verify_attn", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
 _sig("ripe_verify_attn_all_depths", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
 _sig("ripe_verify_attn_all_depths_sliding", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P])
@@ -80,7 +83,7 @@ _sig("ripe_error_string", [_I], ctypes.c_char_p)
 _sig("ripe_last_error", [], ctypes.c_char_p)
 
 EXPORTED = ["ripe_cache_bytes", "ripe_cache_create", "ripe_cache_destroy", "ripe_cache_reset",
-            "ripe_append", "ripe_evict", "ripe_truncate", "ripe_verify_attn",
+            "ripe_append", "ripe_evict", "ripe_truncate", "ripe_fork", "ripe_read_forks", "ripe_verify_attn",
             "ripe_verify_attn_all_depths", "ripe_verify_attn_all_depths_sliding", "ripe_verify_attn_noalloc", "ripe_reserve_workspace",
             "ripe_synth_fill", "ripe_cache_verify_path", "ripe_debug_stall_next_verify", "ripe_accept",
             "ripe_cache_buffers", "ripe_read_meta", "ripe_get_device_error", "ripe_launch_count",
@@ -191,6 +194,20 @@ class RipeCache:
     def ripe_truncate(self, seq_ids: torch.Tensor, new_len: torch.Tensor, stream=None):
         _check(_lib.ripe_truncate(self.handle, _ptr(seq_ids), _ptr(new_len), seq_ids.numel(),
                                   _stream(stream)), "ripe_truncate")
+
+    def ripe_fork(self, parent_ids: torch.Tensor, child_ids: torch.Tensor, stream=None):
+        """Each child becomes a fork of its parent (device int32 ids)."""
+        _check(_lib.ripe_fork(self.handle, _ptr(parent_ids), _ptr(child_ids), parent_ids.numel(),
+                              _stream(stream)), "ripe_fork")
+
+    def ripe_read_forks(self, stream=None):
+        """(fbase, fpos) of every sequence, as host int32 arrays."""
+        import numpy as np
+        fb = np.zeros(self.max_seqs, np.int32)
+        fp = np.zeros(self.max_seqs, np.int32)
+        _check(_lib.ripe_read_forks(self.handle, fb.ctypes.data_as(_P), fp.ctypes.data_as(_P), _stream(stream)),
+               "ripe_read_forks")
+        return fb, fp
 
     def ripe_synth_fill(self, seq_ids, T, seed: int, coef, stream=None):
         """Host lists/arrays: seq_ids, T (per sequence); coef: float[R]."""

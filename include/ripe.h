@@ -70,7 +70,9 @@ enum {
     RIPE_DEVERR_CTX = 4,         /* ctx_len above the committed length; clamped to it */
     RIPE_DEVERR_BRANCH = 5,      /* a branch with depth outside [1,R], rows out of range, more tokens
                                     than the cache's kmax, or a sequence's branches not adjacent */
-    RIPE_DEVERR_TIMEOUT = 6      /* a kernel's bounded wait expired; its outputs are incomplete */
+    RIPE_DEVERR_TIMEOUT = 6,     /* a kernel's bounded wait expired; its outputs are incomplete */
+    RIPE_DEVERR_FORK = 7         /* a fork pair with an id out of range, parent == child, or a parent
+                                    that is itself a fork; that pair was skipped */
 };
 
 /*
@@ -100,6 +102,9 @@ typedef struct {
  *   rfloor[max_seqs] (int32)                           ring floor: the lowest position
  *                 whose ring slots still hold its own planes (rfloor_b <= ws_b);
  *                 append raises it like ws, evict does not
+ *   fbase[max_seqs], fpos[max_seqs] (int32)            forks: sequence b reads its deep
+ *                 positions below fpos_b from sequence fbase_b (b and 0 when b is not
+ *                 a fork)
  * Memory per layer, sequence and head grows as T + W*(R-1) planes instead of R*T
  * (RIPE abstract, sentence on the 64-position window and 11.9% of the full
  * cache's memory).
@@ -124,7 +129,8 @@ int ripe_cache_create(int layers, int R, int H, int d, int W, int Tmax, int max_
 /* Free the cache (and its store if the library allocated it).  Synchronises the device. */
 int ripe_cache_destroy(ripe_cache_t cache);
 
-/* Set len = ws = rfloor = 0 for the listed sequences (device ids, nseq of them). */
+/* Set len = ws = rfloor = 0 for the listed sequences (device ids, nseq of them); a
+ * fork among them is released (it no longer reads its parent). */
 int ripe_cache_reset(ripe_cache_t cache, const int32_t* seq_ids_dev, int nseq,
                      ripe_stream_t stream);
 
@@ -155,6 +161,25 @@ int ripe_append(ripe_cache_t cache, const int32_t* seq_ids_dev, const int32_t* n
  * ring slots below ws become free.
  */
 int ripe_evict(ripe_cache_t cache, const int32_t* seq_ids_dev, int nseq, ripe_stream_t stream);
+
+/*
+ * Branch forks (LoopSpec article, deployment section: the server keeps a KV cache
+ * per branch and deletes rejected continuations).  For each i, sequence
+ * child_ids_dev[i] becomes a fork of parent_ids_dev[i] at the parent's current
+ * length T: it reads the parent's deep plane below its fork position
+ * f = floor(T / 64) * 64 (no copy), owns copies of the parent's deep rows f..T-1
+ * and of the parent's whole ring (Wcap = W + kmax positions x (R-1) planes per
+ * layer and head), and takes the parent's len, ws and rfloor.  Appends, evicts
+ * and verifies of the child then act on the child alone; a verify reads the
+ * parent's prefix and then the child's own positions.  ripe_cache_reset releases
+ * a fork.  While a fork lives its parent must keep its deep rows below f (no
+ * truncate below f) and must not be reset; a fork cannot be truncated below f
+ * (RIPE_DEVERR_COUNT, skipped).  A pair whose parent is itself a fork, whose ids
+ * are out of range or equal, is skipped and sets RIPE_DEVERR_FORK.  Child ids of
+ * one call must be distinct and must not be parents in the same call.
+ */
+int ripe_fork(ripe_cache_t cache, const int32_t* parent_ids_dev, const int32_t* child_ids_dev, int nseq,
+              ripe_stream_t stream);
 
 /*
  * Roll the listed sequences back to a confirmed prefix (LoopSpec article,
@@ -336,6 +361,10 @@ int ripe_debug_stall_next_verify(ripe_cache_t cache, long long cycles);
  * output may be NULL. */
 int ripe_cache_buffers(ripe_cache_t cache, void** kdeep, void** vdeep, void** kwin, void** vwin,
                        int32_t** len, int32_t** ws, int32_t** rfloor);
+
+/* Copy fbase and fpos (fork metadata, see ripe_fork) of all max_seqs sequences to
+ * host arrays (each may be NULL; synchronises stream). */
+int ripe_read_forks(ripe_cache_t cache, int32_t* fbase_host, int32_t* fpos_host, ripe_stream_t stream);
 
 /* Copy len, ws and rfloor of all max_seqs sequences to host arrays (each may be
  * NULL; synchronises stream). */

@@ -44,7 +44,7 @@ def test_cache_bytes_matches_layout_and_memory_model():
     r256 = lambda x: (x + 255) // 256 * 256
     deep = r256(L * B * H * T * d * 2)
     ring = r256(L * B * H * (R - 1) * (W + k) * d * 2)
-    assert n == 2 * deep + 2 * ring + 3 * r256(4 * B) + 256   # len, ws, rfloor, error word
+    assert n == 2 * deep + 2 * ring + 5 * r256(4 * B) + 256   # len, ws, rfloor, fbase, fpos, error word
     # stored planes per (layer, head): T + (W+kmax)(R-1); the live part is T + W(R-1)
     live = T + W * (R - 1)
     assert live / (R * T) == pytest.approx(OR.memory_fraction(T, W, R, 1))

@@ -28,23 +28,33 @@ def compare_store(cache, model, what=""):
     assert np.array_equal(ln, model.length), (what, ln, model.length)
     assert np.array_equal(ws, model.wstart), (what, ws, model.wstart)
     assert np.array_equal(rf, model.rfloor), (what, rf, model.rfloor)
+    fb, fp = cache.ripe_read_forks()
+    assert np.array_equal(fp, model.fpos), (what, fp, model.fpos)
+    assert np.array_equal(fb[fp > 0], model.base[fp > 0]), (what, fb, model.base)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("W", [0, 3, 8])
 def test_append_evict_truncate_bit_exact(dtype, W):
     from depth_planed_kv_b200.ripe import RipeCache
-    L, R, H, d, Tmax, B, kmax = 2, 4, 3, 16, 96, 5, 6
+    L, R, H, d, Tmax, B, kmax = 2, 4, 3, 16, 200, 5, 6
     cache = RipeCache(L, R, H, d, W, Tmax, B, kmax, dtype)
     np_t = np.uint16 if dtype == torch.bfloat16 else np.uint32
     model = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np_t)
     rng = np.random.default_rng(100 + W)
     dev = lambda a: torch.from_numpy(np.asarray(a, np.int32)).cuda()
-    for step in range(40):
-        op = rng.integers(0, 10)
+    for step in range(60):
+        op = rng.integers(0, 11)
         ids = rng.choice(B, size=rng.integers(1, B + 1), replace=False).astype(np.int32)
+        if op == 10:
+            # forks: a parent and a distinct child (sometimes a fork of a fork, flagged)
+            pc = rng.choice(B, size=2, replace=False).astype(np.int32)
+            cache.ripe_fork(dev(pc[:1]), dev(pc[1:]))
+            model.fork(pc[:1], pc[1:])
+            compare_store(cache, model, "step %d fork %s" % (step, pc))
+            continue
         if op < 6:
-            kin = int(rng.choice([1, 2, kmax, 2 * (W + kmax) + 3]))
+            kin = int(rng.choice([1, 2, kmax, 2 * (W + kmax) + 3, 70]))
             n = rng.integers(0, kin + 1, size=len(ids)).astype(np.int32)
             vals = torch.randn(2, L, len(ids), kin, R, H, d).to(dtype).cuda()
             K, V = vals[0].contiguous(), vals[1].contiguous()
