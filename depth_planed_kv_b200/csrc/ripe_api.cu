@@ -126,7 +126,7 @@ int ensure_workspace(ripe_cache_s* c, size_t need, cudaStream_t st) {
         cudaGetLastError();
         return fail(RIPE_ERR_OOM, "cudaMalloc(%zu) for verify scratch failed", sz);
     }
-    // The slice counters at its start must be zero (each call leaves them so).
+    // Zeroed once, so that no partial a kernel skips reads as NaN.
     cudaError_t e = cudaMemset(p, 0, sz);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -154,11 +154,10 @@ int verify_common(ripe_cache_s* c, int layer, const BranchArgs& ba, const void* 
                                         stream_capturing(st));
     if (ba.sliding && !plan.persist)
         return fail(RIPE_ERR_UNSUPPORTED, "the sliding window needs the persistent sm_100a kernel (bf16, d in "
-                    "{64,96,128}, k*R <= 256, R*ceil(k/8) <= %d)", kPersistSlices);
+                    "{64,96,128}, k*R <= 256)");
     int rc = ensure_workspace(c, plan.work_bytes, st);
     if (rc != RIPE_OK) return rc;
-    cudaError_t e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, c->work,
-                                  static_cast<char*>(c->work) + counter_bytes(c), st);
+    cudaError_t e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, c->work, st);
     if (e != cudaSuccess) return cuda_fail(e, "verify launch");
     return RIPE_OK;
 }
@@ -504,12 +503,6 @@ int ripe_get_device_error(ripe_cache_t c, int32_t* code_host, ripe_stream_t stre
     cudaError_t e = cudaMemcpyAsync(code_host, c->err, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(c->err, 0, sizeof(int32_t), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    // A kernel that gave up a wait may have left slice counters mid-count: zero
-    // them so that later calls merge correctly.
-    if (e == cudaSuccess && *code_host == RIPE_DEVERR_TIMEOUT && c->work) {
-        e = cudaMemsetAsync(c->work, 0, counter_bytes(c), st);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    }
     return e == cudaSuccess ? RIPE_OK : cuda_fail(e, "get_device_error");
 }
 

@@ -19,10 +19,6 @@ cudaError_t launch_fork(const ripe_cache_s* c, const int32_t* parents, const int
 cudaError_t launch_synth_fill(const ripe_cache_s* c, int b, int T, uint64_t seed, const float* coef,
                               cudaStream_t st);
 
-// Slice counters of the persistent kernel per (sequence slot, head): one per
-// (depth, 8-token slice) of an all-depths call, so R * ceil(k / 8) <= this.
-constexpr int kPersistSlices = 64;
-
 // Verify plan: how the deep region is split and how much scratch the call needs.
 struct VerifyPlan {
     int nsplit;        // deep-region splits (partials 0..nsplit-1); the window+block partial is nsplit
@@ -37,9 +33,8 @@ struct VerifyPlan {
     int win_ub;        // bound on a branch's window + block keys (CUDA-core kernel)
     // persistent kernel: CTAs, CTAs with deep items, window units per deep / other CTA
     int grid, pd, n_lo, n_hi, ndeep, nunits;
-    size_t cnt_bytes;  // slice counters this call indexes (persistent kernel), else 0
     size_t part_bytes; // per-split partial results
-    size_t work_bytes; // scratch needed: the cache's counter region, then the partials
+    size_t work_bytes; // scratch needed (the partials)
 };
 
 // `capacity`: plan for every length the store can hold (Tmax), not for the host's
@@ -47,9 +42,6 @@ struct VerifyPlan {
 // replay while the sequences grow.
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
                        bool capacity);
-// Bytes of the slice-counter region at the start of a cache's verify scratch (fixed
-// per cache, so calls of any shape lay their partials out after it).
-size_t counter_bytes(const ripe_cache_s* c);
 // True while `st` is being captured into a CUDA graph.
 bool stream_capturing(cudaStream_t st);
 // Re-plan with `nsplit` deep splits (chunk and scratch size follow).
@@ -58,12 +50,13 @@ void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit
 struct VerifyArgs;
 bool fused_supported(int dtype, int d);
 cudaError_t launch_fused(const void* tmaps, const VerifyArgs& a, int gslots, int mt, bool pdl, cudaStream_t st);
-cudaError_t launch_persist(const void* tmaps, const VerifyArgs& a, int32_t* cnt, int pd, int n_lo, int n_hi,
+// The persistent kernel, then the kernel that merges its partials.
+cudaError_t launch_persist(const void* tmaps, const VerifyArgs& a, int pd, int n_lo, int n_hi,
                            int ndeep, int nunits, int grid, int mt, long long probe_cycles, int sliding,
                            int full_box, cudaStream_t st);
 // Window warps of a deep CTA and of another CTA of the persistent kernel (0: no kernel).
 void persist_shape(int d, int mt, int* nww_deep, int* nww_other);
-// The persistent kernel's window units go through its stage ring (one producer warp).
+// The persistent kernel's window units go through its stage ring (producer warps).
 bool persist_ring_ok(int d, int mt, int Wcap, int k, int sliding, int full_box);
 // The fourteen tensor maps of the sm_100a kernels (0 on success).
 int make_tensor_maps(ripe_cache_s* c);
@@ -77,10 +70,10 @@ cudaError_t launch_accept(int nseq, int k, int V, const float* zp, const float* 
                           const int32_t* x2, const float* u, float temperature, int32_t* n_acc, int32_t* token,
                           int32_t* path, cudaStream_t st);
 
-// `cnt`: the slice-counter region (zero between calls); `part`: the partial results.
+// `part`: scratch for the partial results (plan.part_bytes).
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
                           const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,
-                          void* O, float* lse, void* cnt, void* part, cudaStream_t st);
+                          void* O, float* lse, void* part, cudaStream_t st);
 
 // Record a one-line message for ripe_last_error() and return `status`.
 int ripe_fail(int status, const char* fmt, ...);

@@ -79,9 +79,8 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
     ba.max_ntok = c->kmax;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     VerifyPlan plan = plan_verify(c, nbranch, nrows, c->kmax, false, stream_capturing(st));
-    // A branch list never takes the persistent all-depths kernel, so the call
-    // needs only its partial results (no slice counters).  Fewer, longer deep
-    // splits until they fit the fixed array.
+    // A branch list never takes the persistent all-depths kernel.  Fewer, longer
+    // deep splits until the partial results fit the fixed array.
     while (plan.part_bytes > kStaticScratchBytes && plan.nsplit > 1) plan_set_splits(plan, c, nrows, plan.nsplit / 2);
     if (scratch_needed) *scratch_needed = plan.part_bytes;
     if (plan.persist || plan.part_bytes > kStaticScratchBytes)
@@ -91,7 +90,7 @@ extern "C" int ripe_verify_attn_noalloc(ripe_cache_t c, int layer, const ripe_br
     cudaError_t e = static_scratch_address(&work);
     if (e != cudaSuccess)
         return ripe_fail(RIPE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-    e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, nullptr, work, st);
+    e = launch_verify(c, plan, layer, ba, Q, Kb, Vb, ctx, scale, O, lse, work, st);
     if (e != cudaSuccess) return ripe_fail(RIPE_ERR_CUDA, "verify launch: %s", cudaGetErrorString(e));
     return RIPE_OK;
 }

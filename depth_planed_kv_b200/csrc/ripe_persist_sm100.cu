@@ -48,7 +48,6 @@ constexpr int kN = 64;           // deep keys per tile
 constexpr int kDeepWarps = 6;    // warps 0-3 softmax, 4 TMA, 5 MMA
 constexpr int kWR = 8;           // rows per window unit (the N of an m16n8k16 tile)
 constexpr int kMaxItems = 32;    // deep items per CTA
-constexpr int kMaxUnitsPerGroup = kPersistSlices;
 
 // Tensor maps: deep K, V in 64-row boxes (deep region); ring K, V and deep K, V in
 // 8-row boxes (window chunks); Q of this call as [rows][H][d] in 128-row boxes of
@@ -64,7 +63,6 @@ struct DeepItem {
 
 // Scalars of a launch beyond the common verify arguments.
 struct PArgs {
-    int32_t* cnt;      // [nseq][H][kPersistSlices] arrival counters of the 8-row slices (zero between calls)
     int pd;            // CTAs that take deep items
     int n_lo, n_hi;    // window units per deep CTA / per other CTA
     int ndeep;         // G * H * nsplit deep items
@@ -106,13 +104,14 @@ struct PLayout {
     static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_MISC = OFF_WBAR + 2 * NWARPS * 8;
     static constexpr int OFF_ITEMS = OFF_MISC + 64;
-    static constexpr int OFF_FLAGS = OFF_ITEMS + kMaxItems * (int)sizeof(DeepItem);
     // Stage ring: the unit held by each stage.
     static constexpr int DESC_BYTES = 96;
-    static constexpr int OFF_DESC = (OFF_FLAGS + 2 * kMaxUnitsPerGroup + 15) / 16 * 16;
+    static constexpr int OFF_DESC = (OFF_ITEMS + kMaxItems * (int)sizeof(DeepItem) + 15) / 16 * 16;
     // Stage ring: the ticket last issued into each stage.
     static constexpr int OFF_ISS = OFF_DESC + NWARPS * DESC_BYTES;
-    static constexpr int BYTES = OFF_ISS + NWARPS * 4;
+    // Stage ring: whether a stage's last use wrote window rows by 16-byte copies.
+    static constexpr int OFF_DIRTY = OFF_ISS + NWARPS * 4;
+    static constexpr int BYTES = OFF_DIRTY + NWARPS;
     static constexpr int SMEM = BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
@@ -129,22 +128,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 // Named barrier over the four softmax warps (ids 0 is __syncthreads).
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-__device__ __forceinline__ int ld_acquire(const int32_t* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Arrival on a slice counter: release (this thread's earlier writes, and those of
-// the threads it synchronised with at a barrier, are visible to whoever acquires
-// the counter later) and acquire (the partials of earlier arrivals are visible to
-// this thread, and through a later barrier to its CTA).  Returns the old count.
-__device__ __forceinline__ int arrive_acq_rel(int32_t* p) {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
-    return old;
-}
 
 // Context of sequence slot g of an all-depths call: its id, committed length T,
 // deep-region length A and the arrivals E each of its slices expects; ok is
@@ -187,12 +170,6 @@ __device__ __forceinline__ bool slide_visible(int e, int j, int nblk, int ndw, i
     return false;
 }
 
-// Counter of the slice holding row (token j, depth r) of group g, head h.
-__device__ __forceinline__ int32_t* slice_counter(const VerifyArgs& a, const PArgs& p, int g, int j, int r, int h) {
-    const int QS = (a.ba.k + kWR - 1) / kWR;
-    return p.cnt + ((int64_t)g * a.s.H + h) * kPersistSlices + (r - 1) * QS + j / kWR;
-}
-
 template <int D, int MT, int ST, int NWW, int KC, bool RING>
 __global__ void __launch_bounds__(PLayout<D, MT, ST, NWW, KC>::THREADS, 1)
 persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
@@ -229,8 +206,6 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     // Next window unit of this CTA's range to hand to a warp that asks for one.
     int* unit_next = reinterpret_cast<int*>(sm + Lay::OFF_MISC + 16);
     DeepItem* items = reinterpret_cast<DeepItem*>(sm + Lay::OFF_ITEMS);
-    uint8_t* known_last = sm + Lay::OFF_FLAGS;
-    uint8_t* is_last = known_last + kMaxUnitsPerGroup;
 
     const StoreView& s = a.s;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -264,7 +239,10 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             mbar_init(wbar + Lay::NWARPS + i, 1);
         }
         *reinterpret_cast<int*>(sm + Lay::OFF_MISC + 20) = 0;  // the ring's next ticket
-        for (int i = 0; i < Lay::NWARPS; ++i) reinterpret_cast<int*>(sm + Lay::OFF_ISS)[i] = -1;
+        for (int i = 0; i < Lay::NWARPS; ++i) {
+            reinterpret_cast<int*>(sm + Lay::OFF_ISS)[i] = -1;
+            sm[Lay::OFF_DIRTY + i] = 0;
+        }
         *abort_flag = 0;
         const int64_t ub = cta < pa.pd ? (int64_t)cta * pa.n_lo
                                        : (int64_t)pa.pd * pa.n_lo + (int64_t)(cta - pa.pd) * pa.n_hi;
@@ -553,33 +531,20 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     tc_fence_before();
                     mbar_arrive(p_full + sb);
                 }
-                // ---- epilogue of the item.  Slices that already hold every other
-                // arrival are merged here without writing this chunk's partial.
-                const int nslices = R * QS;
-                for (int u = t; u < nslices; u += 128) {
-                    const int r = u / QS + 1, q = u % QS;
-                    known_last[u] = ld_acquire(slice_counter(a, pa, di.g, q * kWR, r, di.h)) == di.E - 1;
-                }
+                // ---- epilogue of the item: publish every row's partial (segment c);
+                // the merge kernel that follows combines the segments.
                 if (ok) ok = warp_wait(pv_done + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, s.err);
                 tc_fence_after();
                 softmax_bar();
-                // Row (token j, depth r) of M row t in tile mt; its slice index.
-                int rows[MT], sl[MT];
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const int rl = mt * 128 + t;
-                    rows[mt] = rl < kR ? grow0 + rl : -1;
-                    sl[mt] = rl < kR ? ((rl % R) * QS + (rl / R) / kWR) : 0;
-                }
-                // Publish the partial of every row whose slice is not known to end here:
                 // 8 rows x 32 columns at a time staged in shared memory, 128-byte pieces.
                 {
                     constexpr int OSTR = 32 * 4 + 16;
                     uint8_t* ostage = sm + Lay::OFF_OST + warp * 8 * OSTR;
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
-                        const bool pub = ok && rows[mt] >= 0 && !known_last[sl[mt]];
-                        const int64_t pi = pub ? ((int64_t)rows[mt] * H + di.h) * a.nseg + di.c : -1;
+                        const int rl = mt * 128 + t;
+                        const bool pub = ok && rl < kR;
+                        const int64_t pi = pub ? ((int64_t)(grow0 + rl) * H + di.h) * a.nseg + di.c : -1;
                         if (pub) a.part_ml[pi] = make_float2(m[mt], l[mt]);
                         if (!__any_sync(0xffffffffu, pub)) continue;
 #pragma unroll 1
@@ -608,85 +573,6 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                             }
                         }
                     }
-                }
-                // The barrier orders every softmax thread's partial writes before the
-                // arrivals; each arrival releases them and acquires the earlier ones.
-                if (t == 0) *stop_snap = *abort_flag;
-                softmax_bar();
-                const bool all_ok = !*stop_snap;
-                for (int u = t; u < nslices; u += 128) {
-                    const int r = u / QS + 1, q = u % QS;
-                    int32_t* cp = slice_counter(a, pa, di.g, q * kWR, r, di.h);
-                    bool last = false;
-                    if (all_ok) {
-                        last = known_last[u];
-                        if (!last) last = arrive_acq_rel(cp) == di.E - 1;
-                        if (last) *cp = 0;  // the last arrival: nothing else touches it in this call
-                    }
-                    is_last[u] = last;
-                }
-                softmax_bar();
-                // Merge the rows of the slices that ended here: this chunk's partial from
-                // TMEM and registers, the other deep chunks' and the window's from scratch.
-                // Segments in the fixed order (deep chunks, then the window) whoever
-                // merges, so the result does not depend on which arrival came last.
-                // tcgen05.ld is warp-collective: a warp loads O when any of its rows
-                // merges, and only those rows use it.
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const bool mine = rows[mt] >= 0 && is_last[sl[mt]];
-                    if (!__any_sync(0xffffffffu, mine)) continue;
-                    const int64_t ro = mine ? (int64_t)rows[mt] * H + di.h : 0;
-                    const int np = mine ? di.E - 1 : 0;  // deep chunks with keys; segment np is the window
-                    float2 ml[9];
-                    float M = -INFINITY;
-                    for (int sg = 0; sg <= np; ++sg) {
-                        ml[sg] = sg == di.c ? make_float2(m[mt], l[mt])
-                                            : __ldcg(a.part_ml + ro * a.nseg + (sg < np ? sg : a.nsplit));
-                        M = fmaxf(M, ml[sg].x);
-                    }
-                    float fs[9], L = 0.f;
-                    for (int sg = 0; sg <= np; ++sg) {
-                        fs[sg] = ex2(ml[sg].x - M);
-                        L = fmaf(ml[sg].y, fs[sg], L);
-                    }
-                    const float inv = 1.f / L;
-                    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        float own[32], acc[32];
-                        tmem_ld32(lane_addr + Lay::O_COL(mt) + c0, own);
-                        tmem_wait_ld();
-                        if (!mine) continue;
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) acc[c] = 0.f;
-                        for (int sg = 0; sg <= np; ++sg) {
-                            const float f = fs[sg];
-                            if (sg == di.c) {
-#pragma unroll
-                                for (int c = 0; c < 32; ++c) acc[c] = fmaf(own[c], f, acc[c]);
-                                continue;
-                            }
-                            const float4* src = reinterpret_cast<const float4*>(
-                                a.part_o + (ro * a.nseg + (sg < np ? sg : a.nsplit)) * D + c0);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const float4 x = __ldcg(src + c);
-                                acc[4 * c] = fmaf(x.x, f, acc[4 * c]);
-                                acc[4 * c + 1] = fmaf(x.y, f, acc[4 * c + 1]);
-                                acc[4 * c + 2] = fmaf(x.z, f, acc[4 * c + 2]);
-                                acc[4 * c + 3] = fmaf(x.w, f, acc[4 * c + 3]);
-                            }
-                        }
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            reinterpret_cast<uint4*>(orow + c0)[c] =
-                                make_uint4(pack_bf16(acc[8 * c] * inv, acc[8 * c + 1] * inv),
-                                           pack_bf16(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
-                                           pack_bf16(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
-                                           pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
-                    }
-                    if (mine && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -763,12 +649,11 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
         struct Slice {
             int g, h, r, j0, nr, E;
         };
-        auto describe = [&](int u) {
+        auto describe_at = [&](int g, int h, int r, int q) {
             Unit w;
-            const int q = u % QS;
-            w.r = (u / QS) % R + 1;
-            w.h = (u / (QS * R)) % H;
-            w.g = u / (QS * R * H);
+            w.r = r;
+            w.h = h;
+            w.g = g;
             if (w.g != cached_g) {
                 gc = group_ctx(a, w.g, false);
                 cached_g = w.g;
@@ -798,6 +683,9 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             w.koff = w.fast ? s.Wcap : w.nw;
             w.nk = w.koff + w.nblk + w.ndw + w.nbr;
             return w;
+        };
+        auto describe = [&](int u) {
+            return describe_at(u / (QS * R * H), (u / (QS * R)) % H, (u / QS) % R + 1, u % QS);
         };
         // The CTA's next unit whose group is valid (warp-uniform).
         auto next_valid = [&](Unit& w) {
@@ -951,75 +839,65 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             finish();
         };
 
-        // The last arrival on a slice merges it: deep chunks in order, then the window
-        // partial, all read back from scratch.  Lane = (row lane/4, float4 column
-        // lane%4 + 4 v); the scale factors first (one round of loads), then the
-        // partials a few segments at a time.  Same arithmetic and order as the deep
-        // merge, so whoever merges writes the same bits.
-        auto resolve = [&](const Slice& w, int old) {
-            const bool last = __shfl_sync(0xffffffffu, old, 0) == w.E - 1;
-            if (!last) return;
-            if (lane == 0) *slice_counter(a, pa, w.g, w.j0, w.r, w.h) = 0;  // nothing else touches it
-            __syncwarp();  // lane 0's acquire, then every lane's reads
-            constexpr int NV = D / 16;
-            const int rr = lane >> 2, c4 = lane & 3;
-            const bool vr = rr < w.nr;
-            const int64_t ro = ((int64_t)w.g * kR + (int64_t)(w.j0 + rr) * R + w.r - 1) * H + w.h;
-            const int np = w.E - 1;  // segment np is the window
-            float2 ml[9];
-            float M = -INFINITY;
-#pragma unroll
-            for (int sg = 0; sg < 9; ++sg) {
-                ml[sg] = make_float2(-INFINITY, 0.f);
-                if (sg <= np && vr) ml[sg] = __ldcg(a.part_ml + ro * a.nseg + (sg < np ? sg : a.nsplit));
-                if (sg <= np) M = fmaxf(M, ml[sg].x);
+        // A whole-window unit into a ring stage: the ring plane (or Wcap deep rows) by
+        // one tensor box per column chunk, the draft tokens after it and the queries
+        // in key rows KC-8.. by 16-byte copies, the rest of the unit's 16-key tiles
+        // zeroed.  Tensor copies write rows below Wcap and the other writes rows from
+        // Wcap on, so a stage needs a proxy fence only after a use that wrote window
+        // rows by copies (a unit of the general form; `dirty`).
+        auto ring_issue = [&](const Unit& w, uint8_t* stage, uint64_t* bar, uint8_t* dirty) {
+            if (*dirty) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) *dirty = 0;
             }
-            float fs[9], L = 0.f;
+            if (lane == 0) {
+                mbar_expect_tx(bar, (uint32_t)(s.Wcap * 64 * NCH * 2));
+                const int64_t y = w.ring ? ((((int64_t)a.layer * s.Bmax + w.seq) * H + w.h) * (R - 1) + (w.r - 1)) * s.Wcap
+                                         : (((int64_t)a.layer * s.Bmax + (w.A < w.fp ? w.fb : w.seq)) * H + w.h) * s.Tmax + w.A;
+                const CUtensorMap* mk = w.ring ? &tm.wkf : &tm.rkf;
+                const CUtensorMap* mv = w.ring ? &tm.wvf : &tm.rvf;
 #pragma unroll
-            for (int sg = 0; sg < 9; ++sg) {
-                fs[sg] = ex2(ml[sg].x - M);
-                if (sg <= np) L = fmaf(ml[sg].y, fs[sg], L);
-            }
-            float4 acc[NV];
-#pragma unroll
-            for (int v = 0; v < NV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-            constexpr int SB = NV >= 6 ? 1 : 2;  // segments per round of loads
-#pragma unroll
-            for (int sb = 0; sb < 9; sb += SB) {
-                if (sb > np) break;
-                float4 x[SB][NV];
-#pragma unroll
-                for (int i = 0; i < SB; ++i) {
-                    const int sg = sb + i;
-                    const float4* src = reinterpret_cast<const float4*>(
-                        a.part_o + (ro * a.nseg + (sg < np ? sg : a.nsplit)) * D);
-#pragma unroll
-                    for (int v = 0; v < NV; ++v)
-                        x[i][v] = (sg <= np && vr) ? __ldcg(src + c4 + 4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int i = 0; i < SB; ++i) {
-                    const int sg = sb + i;
-                    if (sg > np) break;
-                    const float f = fs[sg];
-#pragma unroll
-                    for (int v = 0; v < NV; ++v) {
-                        acc[v].x = fmaf(x[i][v].x, f, acc[v].x);
-                        acc[v].y = fmaf(x[i][v].y, f, acc[v].y);
-                        acc[v].z = fmaf(x[i][v].z, f, acc[v].z);
-                        acc[v].w = fmaf(x[i][v].w, f, acc[v].w);
-                    }
+                for (int c = 0; c < NCH; ++c) {
+                    tma_load_2d(stage + c * Lay::KCB, mk, 32 * c, (int)y, bar);
+                    tma_load_2d(stage + (NCH + c) * Lay::KCB, mv, 32 * c, (int)y, bar);
                 }
             }
-            if (vr) {
-                const float inv = 1.f / L;
-                uint2* orow = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.O) + ro * D);
-#pragma unroll
-                for (int v = 0; v < NV; ++v)
-                    orow[c4 + 4 * v] = make_uint2(pack_bf16(acc[v].x * inv, acc[v].y * inv),
-                                                  pack_bf16(acc[v].z * inv, acc[v].w * inv));
-                if (c4 == 0 && a.lse) a.lse[ro] = (M + log2f(L)) * 0.69314718055994531f;
+            const int64_t grow0 = (int64_t)w.g * kR;
+            // draft tokens e < nblk (K and V rows), then the 8 query rows
+            const int ncopy = (2 * w.nblk + 8) * VPR;
+            for (int e = lane; e < ncopy; e += 32) {
+                const int v = e % VPR, rr = e / VPR, c = v >> 2, v4 = v & 3;
+                const char* src;
+                int kl, part;
+                bool ok = true;
+                if (rr < 2 * w.nblk) {
+                    const int tok = rr >> 1;
+                    part = rr & 1;
+                    src = (part ? a.Vb : a.Kb) + ((grow0 + (int64_t)tok * R + w.r - 1) * H + w.h) * (2 * D) + v * 16;
+                    kl = w.koff + tok;
+                } else {
+                    const int i = rr - 2 * w.nblk;
+                    ok = i < w.nr;
+                    src = a.Q + (ok ? ((grow0 + (int64_t)(w.j0 + i) * R + w.r - 1) * H + w.h) * (2 * D) + v * 16 : 0);
+                    kl = KC - 8 + i;
+                    part = 0;
+                }
+                cp_async16_zfill(stage + (part * NCH + c) * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4), src,
+                                 ok);
             }
+            // zeros in the rows past the unit's keys up to its last 16-key tile (K rows
+            // below the queries', V rows all)
+            const int z0 = w.koff + w.nblk, z1 = (w.nk + 15) / 16 * 16;
+            const int nz = (z1 - z0) * VPR * 2;
+            for (int e = lane; e < nz; e += 32) {
+                const int v = e % VPR, rr = e / VPR, c = v >> 2, v4 = v & 3;
+                const int kl = z0 + (rr >> 1), part = rr & 1;
+                if (part == 1 || kl < KC - 8)
+                    *reinterpret_cast<uint4*>(stage + (part * NCH + c) * Lay::KCB + kl * 64 +
+                                              ((v4 ^ ((kl >> 1) & 3)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            cp_async_mbar_arrive(bar);
         };
 
         // One chunk of keys [k0, k0 + KC) of unit w from the stage at sb_in into the
@@ -1135,8 +1013,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             __syncwarp();  // every lane is done reading the stage
         };
 
-        // Publish a unit's partial (segment nsplit of its rows) and arrive on its
-        // slice; returns lane 0's counter value before the arrival.
+        // Publish a unit's partial (segment nsplit of its rows).
         auto publish = [&](const Slice& w, const float (&o)[NMT][4], float m_a, float m_b, float l_a, float l_b) {
 #pragma unroll
             for (int o2 = 4; o2 < 32; o2 <<= 1) {
@@ -1165,8 +1042,6 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     if (vb) a.part_ml[pb_] = make_float2(m_b, l_b);
                 }
             }
-            __syncwarp();  // orders every lane's partial writes before lane 0's release
-            return lane == 0 ? arrive_acq_rel(slice_counter(a, pa, w.g, w.j0, w.r, w.h)) : 0;
         };
 
         if constexpr (RING) {
@@ -1185,24 +1060,45 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             // memory is one coherent store for the CTA: once the ticket shows, the
             // barrier's earlier phases show too.)
             volatile int* issued = reinterpret_cast<volatile int*>(sm + Lay::OFF_ISS);
-            // Two producer warps (even and odd tickets) where the CTA has the warps.
-            const int NP = (deep_cta ? Lay::NWARPS - kDeepWarps : Lay::NWARPS) >= 4 ? 2 : 1;
+            // Producer warps take tickets in turn: four in a CTA without deep items
+            // (when it has eight warps or more), two or one in a deep CTA.
+            const int nwin = deep_cta ? Lay::NWARPS - kDeepWarps : Lay::NWARPS;
+            const int NP = nwin >= 8 ? 4 : nwin >= 4 ? 2 : 1;
             const int ub = (int)(ub64 < pa.nunits ? ub64 : pa.nunits);
             const int ntk = uend > ub ? uend - ub : 0;
             if (warp >= wfirst && warp < wfirst + NP) {
                 // ---------------------------------------- producers
+                // (g, h, r, q) of the warp's next unit, stepped without divisions
+                const int u0 = ub + (warp - wfirst);
+                int cg = u0 / (QS * R * H), ch = (u0 / (QS * R)) % H, cr = (u0 / QS) % R + 1, cq = u0 % QS;
+                auto step = [&]() {
+                    if (++cq == QS) {
+                        cq = 0;
+                        if (++cr > R) {
+                            cr = 1;
+                            if (++ch == H) {
+                                ch = 0;
+                                ++cg;
+                            }
+                        }
+                    }
+                };
                 for (int idx = warp - wfirst; idx < ntk; idx += NP) {
                     const int st = idx % NS;
                     if (idx >= NS && !warp_wait(empty + st, ((idx / NS) - 1) & 1, abort_flag, s.err)) break;
-                    Unit w = describe(ub + idx);
+                    Unit w = describe_at(cg, ch, cr, cq);
+                    for (int i = 0; i < NP; ++i) step();
                     // every unit here is one chunk with room for its queries
                     if (w.ok && w.nk > KC - 8) {
                         if (lane == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
                         w.ok = false;
                     }
                     if (lane == 0) desc[st] = w;  // published by lane 0's arrival below
-                    if (w.ok) {
+                    if (w.ok && w.fast) {
+                        ring_issue(w, sring + st * Lay::WSTAGE, full + st, sm + Lay::OFF_DIRTY + st);
+                    } else if (w.ok) {
                         issue(w, 0, sring + st * Lay::WSTAGE, full + st, true);
+                        if (lane == 0) sm[Lay::OFF_DIRTY + st] = 1;
                     } else {
                         if (lane == 0) mbar_arrive(full + st);
                         cp_async_mbar_arrive(full + st);
@@ -1214,18 +1110,12 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 cp_async_wait_all();
             } else {
                 // ---------------------------------------- consumers
-                Slice pw;  // the slice whose arrival is looked at next
-                int pold = 0;
-                bool pend = false;
                 while (true) {
                     int t = 0;
                     if (lane == 0) t = atomicAdd(ticket, 1);
                     t = __shfl_sync(0xffffffffu, t, 0);
-                    const bool have = t < ntk;
-                    int old_now = 0;
-                    bool mine = false;
-                    Slice cs{};
-                    if (have) {
+                    if (t >= ntk) break;
+                    {
                         const int st = t % NS;
                         int okc = 1;
                         if (lane == 0) okc = count_wait(issued + st, t - 1, abort_flag, s.err);
@@ -1249,42 +1139,20 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                         }
                         __syncwarp();
                         if (lane == 0) mbar_arrive(empty + st);  // the stage is free again
-                        if (w.ok) {
-                            cs = Slice{w.g, w.h, w.r, w.j0, w.nr, w.E};
-                            old_now = publish(cs, o, m_a, m_b, l_a, l_b);
-                            mine = true;
-                        }
+                        if (w.ok) publish(Slice{w.g, w.h, w.r, w.j0, w.nr, w.E}, o, m_a, m_b, l_a, l_b);
                     }
-                    // The older arrival has returned by now: merge its slice if it was the
-                    // last; after the last ticket, the final arrival too.
-#pragma unroll 1
-                    for (int pass = 0; pass < 2; ++pass) {
-                        if (pend) resolve(pw, pold);
-                        pend = false;
-                        if (mine && pass == 0) {
-                            pw = cs;
-                            pold = old_now;
-                            pend = true;
-                        }
-                        if (have || !pend) break;
-                    }
-                    if (!have) break;
                 }
             }
         } else {
             uint32_t phase = 0;
             bool wok = true;
-            // One site per step (next unit, issue, publish, merge) keeps the loop's code
-            // small.  Each pass: pick the next load (the current unit's next chunk, or a
-            // new unit), issue it, publish and arrive for a unit that just ended, merge
-            // the slice of the arrival before it if that was the last, then wait for
-            // the load and compute on it.
+            // One site per step (next unit, issue, publish) keeps the loop's code small.
+            // Each pass: pick the next load (the current unit's next chunk, or a new
+            // unit), issue it, publish a unit that just ended, then wait for the load
+            // and compute on it.
             Unit cur{};
             int k0 = 0;
             bool started = false;
-            Slice pw;  // the slice whose arrival is looked at next
-            int pold = 0;
-            bool pend = false;
             uint32_t bq[NKS][2];
             float o[NMT][4];
             float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
@@ -1305,27 +1173,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     issue(nxt, nk0, stage, bar, false);
                     if (nk0 == 0) load_q(nxt, bq);  // the current unit's compute is done with bq
                 }
-                int old_now = 0;
-                if (ended) {
-                    const Slice& w = cs;
-                    // ---- publish the unit's partial (segment nsplit) and arrive; whether it
-                    // was the last arrival is looked at when the next unit ends.
-                    old_now = publish(w, o, m_a, m_b, l_a, l_b);
-                }
-                // The older arrival has returned by now: if it was its slice's last, merge
-                // the slice while the next keys are in flight.  After the last unit, the
-                // final arrival is looked at too.
-#pragma unroll 1
-                for (int pass = 0; pass < 2; ++pass) {
-                    if (pend) resolve(pw, pold);
-                    pend = false;
-                    if (ended && pass == 0) {
-                        pw = cs;
-                        pold = old_now;
-                        pend = true;
-                    }
-                    if (have || !pend) break;
-                }
+                if (ended) publish(cs, o, m_a, m_b, l_a, l_b);  // segment nsplit of its rows
                 if (!have) break;
                 cur = nxt;
                 k0 = nk0;
@@ -1366,6 +1214,71 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             if (iss[st] >= 0) mbar_wait(wbar + st, (iss[st] / NS) & 1, &no_abort, s.err);
     }
     if (deep_cta && warp == 5) tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+// The merge of the persistent kernel's partials: one warp per (row, head).  A row
+// of group g has E = (deep splits with keys) + 1 segments: the deep chunks in
+// order, then the window (segment nsplit).  M = max m_s, L = sum l_s 2^(m_s-M),
+// O = sum 2^(m_s-M) o_s / L, lse = (M + log2 L) ln 2, segments in that fixed order.
+template <int D>
+__global__ void __launch_bounds__(256) persist_merge_kernel(VerifyArgs a, int nrows) {
+    sm100::grid_dependency_wait();  // the persistent kernel's partials
+    const int H = a.s.H, kR = a.ba.k * a.s.R;
+    const int lane = threadIdx.x % 32;
+    const int64_t item = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+    if (item >= (int64_t)nrows * H) return;
+    const int row = (int)(item / H), h = (int)(item % H);
+    const GroupCtx gc = group_ctx(a, row / kR, false);
+    if (!gc.ok) return;
+    const int E = gc.E;  // at most nsplit + 1 <= 9
+    const int64_t base = ((int64_t)row * H + h) * a.nseg;
+    float2 ml[9];
+    float M = -INFINITY;
+#pragma unroll
+    for (int sg = 0; sg < 9; ++sg) {
+        ml[sg] = make_float2(-INFINITY, 0.f);
+        if (sg < E) {
+            ml[sg] = __ldcg(a.part_ml + base + (sg < E - 1 ? sg : a.nsplit));
+            M = fmaxf(M, ml[sg].x);
+        }
+    }
+    float L = 0.f;
+    constexpr int NC = D / 32;
+    float acc[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int sg = 0; sg < 9; ++sg) {
+        if (sg < E) {
+            const float f = sm100::ex2(ml[sg].x - M);
+            L = fmaf(ml[sg].y, f, L);
+            const float* po = a.part_o + (base + (sg < E - 1 ? sg : a.nsplit)) * D + lane;
+#pragma unroll
+            for (int i = 0; i < NC; ++i) acc[i] = fmaf(__ldcg(po + 32 * i), f, acc[i]);
+        }
+    }
+    const float inv = 1.f / L;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ((int64_t)row * H + h) * D + lane;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) orow[32 * i] = __float2bfloat16_rn(acc[i] * inv);
+    if (lane == 0 && a.lse) a.lse[(int64_t)row * H + h] = (M + log2f(L)) * 0.69314718055994531f;
+}
+
+template <int D>
+cudaError_t launch_merge(const VerifyArgs& a, int nrows, cudaStream_t st) {
+    const int64_t warps = (int64_t)nrows * a.s.H;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((warps + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, persist_merge_kernel<D>, a, nrows);
+    ripe_count_launch();
+    return e;
 }
 
 template <int D, int MT, int ST, int NWW, int KC, bool RING>
@@ -1426,7 +1339,7 @@ void persist_shape(int d, int mt, int* nww_deep, int* nww_other) {
     *nww_deep = *nww_other = 0;
 }
 
-cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int32_t* cnt, int pd, int n_lo, int n_hi,
+cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int pd, int n_lo, int n_hi,
                            int ndeep, int nunits, int grid, int mt, long long probe_cycles, int sliding,
                            int full_box, cudaStream_t st) {
     // Cache maps: 0 deep K, 1 deep V (64-row boxes); 6 ring K, 7 ring V, 8 deep K,
@@ -1446,14 +1359,19 @@ cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int32_t* c
     tm.rvf = cm[13];
     VerifyArgs a = args;
     if (!make_q_map(&tm.q, a)) return cudaErrorInvalidValue;
-    PArgs pa{cnt, pd, n_lo, n_hi, ndeep, nunits, probe_cycles, sliding, full_box};
+    PArgs pa{pd, n_lo, n_hi, ndeep, nunits, probe_cycles, sliding, full_box};
     const int d = a.s.d;
     // The stage ring when every unit is one chunk with room for its queries.
     const bool ring = persist_ring_ok(d, mt, a.s.Wcap, a.ba.k, sliding, full_box);
-#define RIPE_LAUNCH(D_, MT_, ST_, NWW_, KC_)                                              \
-    if (d == D_ && mt == MT_)                                                          \
-        return ring ? launch_p<D_, MT_, ST_, NWW_, KC_, true>(tm, a, pa, grid, st)      \
-                    : launch_p<D_, MT_, ST_, NWW_, KC_, false>(tm, a, pa, grid, st);
+    // The kernel publishes every partial; the merge kernel (its dependent launch)
+    // combines them.
+#define RIPE_LAUNCH(D_, MT_, ST_, NWW_, KC_)                                                 \
+    if (d == D_ && mt == MT_) {                                                           \
+        cudaError_t e = ring ? launch_p<D_, MT_, ST_, NWW_, KC_, true>(tm, a, pa, grid, st)  \
+                             : launch_p<D_, MT_, ST_, NWW_, KC_, false>(tm, a, pa, grid, st); \
+        if (e != cudaSuccess) return e;                                                   \
+        return launch_merge<D_>(a, a.ba.nrows, st);                                       \
+    }
     RIPE_LAUNCH(64, 1, 4, 6, 80)
     RIPE_LAUNCH(96, 1, 4, 4, 80)
     RIPE_LAUNCH(128, 1, 3, 3, 80)

@@ -405,7 +405,7 @@ bool plan_persist(const ripe_cache_s* c, int nseq, int k, int len_ub, VerifyPlan
     const int A_ub = len_ub - c->W > 0 ? len_ub - c->W : 0;
     const int R = c->R, H = c->H, d = c->d;
     const int kR = k * R, QS = (k + 7) / 8;
-    if (kR > 256 || R * QS > kPersistSlices || nseq < 1) return false;
+    if (kR > 256 || nseq < 1) return false;
     const int mt = kR > 128 ? 2 : 1;
     int nww_deep = 0, nww_other = 0;
     persist_shape(d, mt, &nww_deep, &nww_other);
@@ -467,7 +467,6 @@ bool plan_persist(const ripe_cache_s* c, int nseq, int k, int len_ub, VerifyPlan
     p.nunits = (int)NU;
     p.mt = mt;
     p.persist = true;
-    p.cnt_bytes = (size_t)nseq * H * kPersistSlices * sizeof(int32_t);
     return true;
 }
 
@@ -485,10 +484,6 @@ int device_sm_count() {
     return count[dev];
 }
 
-size_t counter_bytes(const ripe_cache_s* c) {
-    return ((size_t)c->Bmax * c->H * kPersistSlices * sizeof(int32_t) + 255) / 256 * 256;
-}
-
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
                        bool capacity) {
     VerifyPlan p{};
@@ -502,7 +497,7 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
     p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
     if (p.fused && all_depths && plan_persist(c, nbranch / c->R, max_ntok, len_ub, p)) {
         p.part_bytes = verify_work_bytes(nrows, c->H, c->d, p.nsplit + 1);
-        p.work_bytes = counter_bytes(c) + p.part_bytes;
+        p.work_bytes = p.part_bytes;
         return p;
     }
     int64_t ns;
@@ -536,14 +531,13 @@ void plan_set_splits(VerifyPlan& p, const ripe_cache_s* c, int nrows, int nsplit
     int chunk = (A_ub + nsplit - 1) / nsplit;
     chunk = (chunk + align - 1) / align * align;
     p.chunk = chunk < align ? align : chunk;
-    p.cnt_bytes = 0;
     p.part_bytes = verify_work_bytes(nrows, c->H, c->d, nsplit + 1);
-    p.work_bytes = counter_bytes(c) + p.part_bytes;
+    p.work_bytes = p.part_bytes;
 }
 
 cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int layer, const BranchArgs& ba,
                           const void* Q, const void* Kb, const void* Vb, const int32_t* ctx, float scale,
-                          void* O, float* lse, void* cnt, void* work, cudaStream_t st) {
+                          void* O, float* lse, void* work, cudaStream_t st) {
     VerifyArgs a;
     a.s = store_view(c);
     a.ba = ba;
@@ -562,7 +556,7 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     if (plan.persist) {
         // The test hook is consumed by the launch it applies to.
         const long long probe = const_cast<ripe_cache_s*>(c)->probe_cycles.exchange(0);
-        e = launch_persist(c->tmaps, a, reinterpret_cast<int32_t*>(cnt), plan.pd, plan.n_lo, plan.n_hi, plan.ndeep,
+        e = launch_persist(c->tmaps, a, plan.pd, plan.n_lo, plan.n_hi, plan.ndeep,
                            plan.nunits, plan.grid, plan.mt, probe, ba.sliding, c->full_box ? 1 : 0, st);
         if (e != cudaSuccess) return e;
     } else if (plan.fused) {

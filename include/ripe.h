@@ -248,8 +248,8 @@ int ripe_verify_attn_all_depths(ripe_cache_t cache, int layer, const int32_t* se
  * read at plane R, which is its depth-R row in the same call.  With W >= k no
  * draft token is read at plane R (batched verification is then block-independent).
  * Same arguments and layouts as ripe_verify_attn_all_depths.  Served by the
- * persistent sm_100a kernel only (bf16, d in {64, 96, 128}, k*R <= 256 and
- * R*ceil(k/8) <= 64); RIPE_ERR_UNSUPPORTED otherwise.
+ * persistent sm_100a kernel only (bf16, d in {64, 96, 128}, k*R <= 256);
+ * RIPE_ERR_UNSUPPORTED otherwise.
  */
 int ripe_verify_attn_all_depths_sliding(ripe_cache_t cache, int layer, const int32_t* seq_ids_dev, int nseq,
                                         int k, const void* Q, const void* Kblk, const void* Vblk,
@@ -352,8 +352,8 @@ int ripe_accept(int nseq, int k, int V, const float* zp, const float* zq, const 
  * <= 2^31; 0 turns the hook off), on a barrier that nothing signals.  The wait runs
  * out, the kernel records RIPE_DEVERR_TIMEOUT, lets its copies and tensor-core
  * operations in flight finish, and returns with that call's outputs incomplete;
- * ripe_get_device_error then reports it and clears the merge counters, and later
- * calls are exact again.  No fault, trap or unbounded wait is involved.
+ * ripe_get_device_error then reports it, and later calls are exact again.  No
+ * fault, trap or unbounded wait is involved.
  */
 int ripe_debug_stall_next_verify(ripe_cache_t cache, long long cycles);
 
