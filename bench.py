@@ -314,6 +314,7 @@ class Work:
         self.host_in, self.dev_in, self.outs, self.outs_host = [], [], [], []
         self.post = None
         self.steps = None        # fixed timed step count (None: --steps)
+        self.warmup = None       # fixed warm-up count (None: --warmup, at least 3)
         self.preroll = True      # run ~1 s of untimed steps first (identical, store unchanged)
         self.verify_events = False  # time each verify inside the timed region (roofline)
         self.extra = {}
@@ -473,7 +474,10 @@ def make_long_work(rank, peaks):
 
     wk.call = call
     wk.post = post
+    # The store holds Tmax = ctx + 512 positions and a step appends up to 8 tokens per
+    # sequence: 3 warm-up + 16 timed steps, then 3 + 16 more end to end, is 38 <= 64.
     wk.steps = 16
+    wk.warmup = 3
     wk.preroll = False
     wk.verify_events = True
     # bytes of a step: the verify's, plus the append's (read the accepted tokens'
@@ -492,7 +496,7 @@ def run_work(wk, args, world, rank, local, peaks, peak_kind):
     from depth_planed_kv_b200.ripe import launch_count
     stream = torch.cuda.current_stream()
     steps = wk.steps or args.steps
-    warmup = max(args.warmup, 3)
+    warmup = wk.warmup or max(args.warmup, 3)
 
     def barrier():
         torch.cuda.synchronize()
@@ -561,7 +565,7 @@ def run_work(wk, args, world, rank, local, peaks, peak_kind):
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_for(wk.config["workload"]),
             "peak_source": peak_kind,
-            "kernel": "the verify kernel (one launch per ripe_verify_attn* call); CUDA events on its stream"}
+            "kernel": "the verify call: the persistent kernel and its merge kernel (one ripe_verify_attn* call); CUDA events on their stream"}
     if isolated is not None:
         roof["isolated_call_us"] = isolated
     clocks = dict(sampler.summary(), window="1 s of identical steps before and through the timed region"

@@ -1085,7 +1085,14 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 };
                 for (int idx = warp - wfirst; idx < ntk; idx += NP) {
                     const int st = idx % NS;
-                    if (idx >= NS && !warp_wait(empty + st, ((idx / NS) - 1) & 1, abort_flag, s.err)) break;
+                    if (idx >= NS) {
+                        // The stage's previous ticket (another producer's) must be issued
+                        // before its empty barrier is looked at, for the same reason.
+                        int okc = 1;
+                        if (lane == 0) okc = count_wait(issued + st, idx - NS - 1, abort_flag, s.err);
+                        if (!__shfl_sync(0xffffffffu, okc, 0)) break;
+                        if (!warp_wait(empty + st, ((idx / NS) - 1) & 1, abort_flag, s.err)) break;
+                    }
                     Unit w = describe_at(cg, ch, cr, cq);
                     for (int i = 0; i < NP; ++i) step();
                     // every unit here is one chunk with room for its queries

@@ -393,8 +393,7 @@ cudaError_t launch_seg(const VerifyArgs& a, int seg_first, int seg_count, int nb
 }
 
 // The persistent kernel serves an all-depths call whose k*R rows of a sequence
-// fit two 128-row M tiles and whose (depth, 8-token) slices fit the counter
-// layout.  The plan splits the deep region into nsplit chunks and balances the
+// fit two 128-row M tiles.  The plan splits the deep region into nsplit chunks and balances the
 // bytes each CTA streams: pd CTAs take deep items (sequence, head, chunk) pd
 // apart plus n_lo window units each; the others take n_hi window units.  A deep
 // item also costs a fixed latency (Q load, pipeline fill, epilogue), counted as
@@ -414,7 +413,11 @@ bool plan_persist(const ripe_cache_s* c, int nseq, int k, int len_ub, VerifyPlan
     if (P < 1) return false;
     const double kv = 4.0 * d, row = 2.0 * d;
     const int wl = len_ub < c->W ? len_ub : c->W;
-    const double bU = (wl + k) * kv + 2.0 * (k < 8 ? k : 8) * row;
+    // A window unit costs its bytes, but at least a fixed ~20 KB-equivalent of issue
+    // and compute time (measured: a unit of a few KB takes about as long as one
+    // of 20 KB).
+    const double bU_bytes = (wl + k) * kv + 2.0 * (k < 8 ? k : 8) * row;
+    const double bU = bU_bytes > 20e3 ? bU_bytes : 20e3;
     const double item_fixed = 96e3;
     const int64_t NU = (int64_t)nseq * H * R * QS;
     if (NU > (1 << 30)) return false;

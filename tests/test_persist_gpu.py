@@ -71,3 +71,11 @@ def test_context_override_and_repeats():
     wl = S.Workload("p_ctx", 1, 32, 4, 96, 64, 4, 3, None, 0.88, 1205, "bf16", 1200, 4)
     ctx = np.array([1100, 500, 64])
     _verify_and_check(wl, ctx, ctx_len=np.array([900, 500, 30]), reps=3)
+
+
+@pytest.mark.parametrize("W", [0, 4])
+def test_many_window_units_per_cta(W):
+    # The 55-head, 32-depth shape with a small window: the planner puts many window
+    # units on each CTA, so the stage ring's producer warps run far apart.
+    wl = S.Workload("p_units_w%d" % W, 1, 32, 55, 96, W, 4, 1, None, 0.88, 1206, "bf16", 1088, 4)
+    _verify_and_check(wl, np.array([1024]), heads=[0, 17, 54], reps=2)
