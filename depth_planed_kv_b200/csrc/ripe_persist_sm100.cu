@@ -10,30 +10,35 @@
 //
 // Work items, spread over one wave of CTAs (one CTA per SM):
 //   deep item (sequence g, head h, chunk c): keys [c*chunk, (c+1)*chunk) of the
-//     deep region for all k*R rows (the last chunk runs to the region's end).  S = Q K^T (tcgen05.mma, fp32 in TMEM), online
+//     deep region for all k*R rows (the last chunk runs to the region's end).
+//     S = Q K^T (tcgen05.mma, fp32 in TMEM), online
 //     softmax on CUDA cores, O += P V (tcgen05.mma, P read from TMEM); K, V by TMA
 //     through ST shared-memory stages.  Warps 0-3 own TMEM lanes (one row each),
 //     warp 4 lane 0 issues TMA, warp 5 allocates TMEM and its lane 0 issues MMAs.
 //     The first `pd` CTAs take deep items pd apart.
 //   window unit (g, h, r, 8-token slice q): the window keys at plane r (ring
-//     slots, or deep-plane rows for r = R) and the slice's draft-block keys, in
-//     chunks of KC keys.  One warp runs a unit: it loads a chunk into its own
-//     shared-memory stage (8-row TMA boxes where eight window keys sit contiguously
-//     in memory, 16-byte cp.async for the rest and for block keys), then
+//     slots, or deep-plane rows for r = R) and the slice's draft-block keys, then
 //     S^T = K Q^T and O^T = V^T P^T on warp-level MMA tiles (m16n8k16: keys and
 //     channels on the 16-row side, the <= 8 query rows on the 8-column side).
 //     Every CTA takes a contiguous range of units: n_lo per deep CTA, n_hi per
-//     other CTA (the host balances the bytes).  A CTA without deep items turns
-//     its deep warps and deep stages into more window warps.
+//     other CTA (the host balances the work).  Two forms:
+//     * stage ring (every unit one chunk of KC keys, no sliding window): producer
+//       warps load units in order into a ring of shared-memory stages (the whole
+//       ring plane by one Wcap-row tensor box per column chunk, the draft tokens by
+//       16-byte copies); consumer warps (the deep warps too, once their items are
+//       done) take tickets, compute, free the stage and publish.  A consumer loads
+//       the queries of its next unit into registers while it computes this one.
+//     * per-warp stages (otherwise): each warp runs its units one chunk at a time
+//       through its own stage (8-row boxes where eight window keys sit together in
+//       memory, copies for the rest).
 //
-// Merge without waiting: every item and unit that finishes leaves its partial
-// result (m in log2 units, l, unnormalised o) in scratch, then arrives on the
-// counter of each 8-row slice it covered.  A slice expects one arrival per deep
-// chunk that holds keys plus one from its window unit; the last arrival combines
-// the slice's partials -- M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L --
-// writes O and the LSE, and resets the counter to zero for the next call.  An
-// arrival that sees it will be last (the counter already holds every other
-// arrival) skips writing its own partial.  No CTA ever waits for another.
+// No merging here: every deep item and window unit writes its partial result (m
+// in log2 units, l, unnormalised o) to scratch -- segment c of its rows for deep
+// chunk c, segment nsplit for the window -- and the merge kernel launched after
+// this one (programmatic dependent launch) combines each row's segments in fixed
+// order: M = max m, L = sum l 2^(m-M), O = sum o 2^(m-M) / L, and the LSE.  No CTA
+// ever waits for another; global round trips under full memory load cost
+// microseconds, so the kernel makes none on its critical paths.
 #include <cuda.h>
 
 #include <cstring>
@@ -658,6 +663,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 gc = group_ctx(a, w.g, false);
                 cached_g = w.g;
             }
+            // The group's segment count for the merge kernel, from its first unit.
+            if (h == 0 && r == 1 && q == 0 && lane == 0) a.gE[g] = gc.ok ? gc.E : 0;
             w.ok = gc.ok;
             w.E = gc.E;
             w.A = gc.A;
@@ -713,7 +720,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
         // contiguous in memory by TMA (lane 0), the rest (a group that wraps the ring,
         // a partial group, draft tokens, plane-R keys of the sliding window, zero fill)
         // by 16-byte copies.  The stage's earlier reads are done (caller's __syncwarp).
-        auto issue = [&](const Unit& w, int k0, uint8_t* stage, uint64_t* bar, bool qrows) {
+        auto issue = [&](const Unit& w, int k0, uint8_t* stage, uint64_t* bar) {
             const int nt = (min(KC, w.nk - k0) + 15) / 16;
             const int64_t grow0 = (int64_t)w.g * kR;
             // Rows of ring plane r (slot 0) and of the deep plane (position 0; deep_yp:
@@ -763,24 +770,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 const bool valid = key_src(k0 + kl, v, ks_, vs_);
                 const int c = v >> 2, v4 = v & 3;
                 uint8_t* dk = stage + c * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4);
-                if (!qrows || kl < KC - 8) cp_async16_zfill(dk, ks_, valid);  // else the row holds Q
+                cp_async16_zfill(dk, ks_, valid);
                 cp_async16_zfill(dk + NCH * Lay::KCB, vs_, valid);
-            };
-            // The slice's query rows (zeros past nr) into key rows KC-8.. of the K part.
-            auto finish = [&]() {
-                if (qrows) {
-                    const int64_t grow0q = (int64_t)w.g * kR;
-                    for (int e = lane; e < 8 * VPR; e += 32) {
-                        const int i = e / VPR, v = e % VPR, kl = KC - 8 + i;
-                        const bool okq = i < w.nr;
-                        const char* qs = a.Q + (okq ? ((grow0q + (int64_t)(w.j0 + i) * R + w.r - 1) * H + w.h) *
-                                                              (2 * D) + v * 16
-                                                        : 0);
-                        const int c = v >> 2, v4 = v & 3;
-                        cp_async16_zfill(stage + c * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4), qs, okq);
-                    }
-                }
-                cp_async_mbar_arrive(bar);
             };
             if (w.fast) {
                 // The whole window in one box per column chunk (k0 = 0), then the
@@ -798,7 +789,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 }
                 const int nrest = 16 * nt - s.Wcap;
                 for (int e = lane; e < nrest * VPR; e += 32) copy_key(s.Wcap + e / VPR, e % VPR);
-                finish();
+                cp_async_mbar_arrive(bar);
                 return;
             }
             uint32_t tma_groups = 0;
@@ -836,13 +827,12 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 other &= other - 1;
                 for (int e = lane; e < 8 * VPR; e += 32) copy_key(8 * gm + e / VPR, e % VPR);
             }
-            finish();
+            cp_async_mbar_arrive(bar);
         };
 
         // A whole-window unit into a ring stage: the ring plane (or Wcap deep rows) by
-        // one tensor box per column chunk, the draft tokens after it and the queries
-        // in key rows KC-8.. by 16-byte copies, the rest of the unit's 16-key tiles
-        // zeroed.  Tensor copies write rows below Wcap and the other writes rows from
+        // one tensor box per column chunk (a lane each), the draft tokens after it by
+        // 16-byte copies, the V rows of the rest of the unit's 16-key tiles zeroed.  Tensor copies write rows below Wcap and the other writes rows from
         // Wcap on, so a stage needs a proxy fence only after a use that wrote window
         // rows by copies (a unit of the general form; `dirty`).
         auto ring_issue = [&](const Unit& w, uint8_t* stage, uint64_t* bar, uint8_t* dirty) {
@@ -851,51 +841,35 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 __syncwarp();
                 if (lane == 0) *dirty = 0;
             }
-            if (lane == 0) {
-                mbar_expect_tx(bar, (uint32_t)(s.Wcap * 64 * NCH * 2));
+            if (lane == 0) mbar_expect_tx(bar, (uint32_t)(s.Wcap * 64 * NCH * 2));
+            __syncwarp();
+            if (lane < 2 * NCH) {  // one box per lane: K column chunks, then V
                 const int64_t y = w.ring ? ((((int64_t)a.layer * s.Bmax + w.seq) * H + w.h) * (R - 1) + (w.r - 1)) * s.Wcap
                                          : (((int64_t)a.layer * s.Bmax + (w.A < w.fp ? w.fb : w.seq)) * H + w.h) * s.Tmax + w.A;
-                const CUtensorMap* mk = w.ring ? &tm.wkf : &tm.rkf;
-                const CUtensorMap* mv = w.ring ? &tm.wvf : &tm.rvf;
-#pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                    tma_load_2d(stage + c * Lay::KCB, mk, 32 * c, (int)y, bar);
-                    tma_load_2d(stage + (NCH + c) * Lay::KCB, mv, 32 * c, (int)y, bar);
-                }
+                const bool isv = lane >= NCH;
+                const int c = isv ? lane - NCH : lane;
+                const CUtensorMap* m = w.ring ? (isv ? &tm.wvf : &tm.wkf) : (isv ? &tm.rvf : &tm.rkf);
+                tma_load_2d(stage + lane * Lay::KCB, m, 32 * c, (int)y, bar);
             }
             const int64_t grow0 = (int64_t)w.g * kR;
-            // draft tokens e < nblk (K and V rows), then the 8 query rows
-            const int ncopy = (2 * w.nblk + 8) * VPR;
+            // draft tokens e < nblk (K and V rows)
+            const int ncopy = 2 * w.nblk * VPR;
             for (int e = lane; e < ncopy; e += 32) {
                 const int v = e % VPR, rr = e / VPR, c = v >> 2, v4 = v & 3;
-                const char* src;
-                int kl, part;
-                bool ok = true;
-                if (rr < 2 * w.nblk) {
-                    const int tok = rr >> 1;
-                    part = rr & 1;
-                    src = (part ? a.Vb : a.Kb) + ((grow0 + (int64_t)tok * R + w.r - 1) * H + w.h) * (2 * D) + v * 16;
-                    kl = w.koff + tok;
-                } else {
-                    const int i = rr - 2 * w.nblk;
-                    ok = i < w.nr;
-                    src = a.Q + (ok ? ((grow0 + (int64_t)(w.j0 + i) * R + w.r - 1) * H + w.h) * (2 * D) + v * 16 : 0);
-                    kl = KC - 8 + i;
-                    part = 0;
-                }
-                cp_async16_zfill(stage + (part * NCH + c) * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4), src,
-                                 ok);
+                const int tok = rr >> 1, part = rr & 1, kl = w.koff + tok;
+                const char* src =
+                    (part ? a.Vb : a.Kb) + ((grow0 + (int64_t)tok * R + w.r - 1) * H + w.h) * (2 * D) + v * 16;
+                cp_async16(stage + (part * NCH + c) * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4), src);
             }
-            // zeros in the rows past the unit's keys up to its last 16-key tile (K rows
-            // below the queries', V rows all)
+            // zeros in the V rows past the unit's keys up to its last 16-key tile (their
+            // probabilities are 0, and 0 x finite is 0; K rows there are masked whatever
+            // they hold)
             const int z0 = w.koff + w.nblk, z1 = (w.nk + 15) / 16 * 16;
-            const int nz = (z1 - z0) * VPR * 2;
+            const int nz = (z1 - z0) * VPR;
             for (int e = lane; e < nz; e += 32) {
-                const int v = e % VPR, rr = e / VPR, c = v >> 2, v4 = v & 3;
-                const int kl = z0 + (rr >> 1), part = rr & 1;
-                if (part == 1 || kl < KC - 8)
-                    *reinterpret_cast<uint4*>(stage + (part * NCH + c) * Lay::KCB + kl * 64 +
-                                              ((v4 ^ ((kl >> 1) & 3)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                const int v = e % VPR, kl = z0 + e / VPR, c = v >> 2, v4 = v & 3;
+                *reinterpret_cast<uint4*>(stage + (NCH + c) * Lay::KCB + kl * 64 + ((v4 ^ ((kl >> 1) & 3)) << 4)) =
+                    make_uint4(0u, 0u, 0u, 0u);
             }
             cp_async_mbar_arrive(bar);
         };
@@ -1095,8 +1069,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     }
                     Unit w = describe_at(cg, ch, cr, cq);
                     for (int i = 0; i < NP; ++i) step();
-                    // every unit here is one chunk with room for its queries
-                    if (w.ok && w.nk > KC - 8) {
+                    // every unit here is one chunk
+                    if (w.ok && w.nk > KC) {
                         if (lane == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
                         w.ok = false;
                     }
@@ -1104,7 +1078,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     if (w.ok && w.fast) {
                         ring_issue(w, sring + st * Lay::WSTAGE, full + st, sm + Lay::OFF_DIRTY + st);
                     } else if (w.ok) {
-                        issue(w, 0, sring + st * Lay::WSTAGE, full + st, true);
+                        issue(w, 0, sring + st * Lay::WSTAGE, full + st);
                         if (lane == 0) sm[Lay::OFF_DIRTY + st] = 1;
                     } else {
                         if (lane == 0) mbar_arrive(full + st);
@@ -1117,37 +1091,52 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 cp_async_wait_all();
             } else {
                 // ---------------------------------------- consumers
-                while (true) {
+                // A consumer claims its next ticket as it starts a unit and loads that
+                // unit's queries into registers meanwhile (the ticket names the unit).
+                auto claim = [&](uint32_t (&b)[NKS][2]) {
                     int t = 0;
                     if (lane == 0) t = atomicAdd(ticket, 1);
                     t = __shfl_sync(0xffffffffu, t, 0);
-                    if (t >= ntk) break;
-                    {
-                        const int st = t % NS;
-                        int okc = 1;
-                        if (lane == 0) okc = count_wait(issued + st, t - 1, abort_flag, s.err);
-                        if (!__shfl_sync(0xffffffffu, okc, 0)) break;
-                        if (!warp_wait(full + st, (t / NS) & 1, abort_flag, s.err)) break;
-                        const Unit w = desc[st];
-                        const uint32_t sa = smem_u32(sring + st * Lay::WSTAGE);
-                        float o[NMT][4];
-                        float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-                        if (w.ok) {
-                            // Q^T fragments from the stage's last 8 key rows of each column chunk
-                            uint32_t bq[NKS][2];
-                            const int qr = KC - 8 + (lane & 7);
-#pragma unroll
-                            for (int c = 0; c < NCH; ++c)
-                                ldsm_x4_r(smem_ready(sa) + c * Lay::KCB + qr * 64 + (((lane >> 3) ^ ((qr >> 1) & 3)) << 4),
-                                          bq[2 * c][0], bq[2 * c][1], bq[2 * c + 1][0], bq[2 * c + 1][1]);
-#pragma unroll
-                            for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-                            compute(w, 0, sa, bq, o, m_a, m_b, l_a, l_b);
-                        }
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(empty + st);  // the stage is free again
-                        if (w.ok) publish(Slice{w.g, w.h, w.r, w.j0, w.nr, w.E}, o, m_a, m_b, l_a, l_b);
+                    if (t < ntk) {
+                        const int u = ub + t;
+                        Unit q;
+                        q.g = u / (QS * R * H);
+                        q.h = (u / (QS * R)) % H;
+                        q.r = (u / QS) % R + 1;
+                        q.j0 = (u % QS) * kWR;
+                        q.nr = min(kWR, k - q.j0);
+                        load_q(q, b);
                     }
+                    return t;
+                };
+                uint32_t bqn[NKS][2];
+                int tn = claim(bqn);
+                while (tn < ntk) {
+                    const int t = tn;
+                    uint32_t bq[NKS][2];
+#pragma unroll
+                    for (int ks = 0; ks < NKS; ++ks) {
+                        bq[ks][0] = bqn[ks][0];
+                        bq[ks][1] = bqn[ks][1];
+                    }
+                    tn = claim(bqn);
+                    const int st = t % NS;
+                    int okc = 1;
+                    if (lane == 0) okc = count_wait(issued + st, t - 1, abort_flag, s.err);
+                    if (!__shfl_sync(0xffffffffu, okc, 0)) break;
+                    if (!warp_wait(full + st, (t / NS) & 1, abort_flag, s.err)) break;
+                    const Unit w = desc[st];
+                    const uint32_t sa = smem_u32(sring + st * Lay::WSTAGE);
+                    float o[NMT][4];
+                    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+                    if (w.ok) {
+#pragma unroll
+                        for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+                        compute(w, 0, sa, bq, o, m_a, m_b, l_a, l_b);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty + st);  // the stage is free again
+                    if (w.ok) publish(Slice{w.g, w.h, w.r, w.j0, w.nr, w.E}, o, m_a, m_b, l_a, l_b);
                 }
             }
         } else {
@@ -1177,7 +1166,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                 }
                 const bool ended = started && nk0 == 0;
                 if (have) {
-                    issue(nxt, nk0, stage, bar, false);
+                    issue(nxt, nk0, stage, bar);
                     if (nk0 == 0) load_q(nxt, bq);  // the current unit's compute is done with bq
                 }
                 if (ended) publish(cs, o, m_a, m_b, l_a, l_b);  // segment nsplit of its rows
@@ -1223,46 +1212,81 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     if (deep_cta && warp == 5) tmem_dealloc(tmem, Lay::TMEM_COLS);
 }
 
-// The merge of the persistent kernel's partials: one warp per (row, head).  A row
-// of group g has E = (deep splits with keys) + 1 segments: the deep chunks in
-// order, then the window (segment nsplit).  M = max m_s, L = sum l_s 2^(m_s-M),
-// O = sum 2^(m_s-M) o_s / L, lse = (M + log2 L) ln 2, segments in that fixed order.
+// The merge of the persistent kernel's partials: one warp per (row, head), small
+// enough that every warp of the grid is resident at once.  A row of group g has
+// E = gE[g] segments (0: the group was skipped): deep chunks 0..E-2 in order, then
+// the window (segment nsplit).  M = max m_s, L = sum l_s 2^(m_s-M),
+// O = sum 2^(m_s-M) o_s / L, lse = (M + log2 L) ln 2, segments in that order.
+// E and the first segments load together (the deep ones speculatively).
 template <int D>
-__global__ void __launch_bounds__(256) persist_merge_kernel(VerifyArgs a, int nrows) {
+__global__ void __launch_bounds__(128, 12) persist_merge_kernel(VerifyArgs a, int nrows) {
     sm100::grid_dependency_wait();  // the persistent kernel's partials
     const int H = a.s.H, kR = a.ba.k * a.s.R;
     const int lane = threadIdx.x % 32;
-    const int64_t item = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+    const int64_t item = (int64_t)blockIdx.x * 4 + threadIdx.x / 32;
     if (item >= (int64_t)nrows * H) return;
     const int row = (int)(item / H), h = (int)(item % H);
-    const GroupCtx gc = group_ctx(a, row / kR, false);
-    if (!gc.ok) return;
-    const int E = gc.E;  // at most nsplit + 1 <= 9
+    const int E = __ldcg(a.gE + row / kR);
     const int64_t base = ((int64_t)row * H + h) * a.nseg;
-    float2 ml[9];
-    float M = -INFINITY;
+    constexpr int NC = D / 32, NS0 = 3;  // deep segments loaded with E
+    const int nd0 = a.nsplit < NS0 ? a.nsplit : NS0;
+    float2 mw = __ldcg(a.part_ml + base + a.nsplit);
+    float xw[NC];
+    {
+        const float* po = a.part_o + (base + a.nsplit) * D + lane;
 #pragma unroll
-    for (int sg = 0; sg < 9; ++sg) {
-        ml[sg] = make_float2(-INFINITY, 0.f);
-        if (sg < E) {
-            ml[sg] = __ldcg(a.part_ml + base + (sg < E - 1 ? sg : a.nsplit));
-            M = fmaxf(M, ml[sg].x);
+        for (int i = 0; i < NC; ++i) xw[i] = __ldcg(po + 32 * i);
+    }
+    float2 md[NS0];
+    float xd[NS0][NC];
+#pragma unroll
+    for (int j = 0; j < NS0; ++j) {
+        md[j] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+        for (int i = 0; i < NC; ++i) xd[j][i] = 0.f;
+        if (j < nd0) {
+            md[j] = __ldcg(a.part_ml + base + j);
+            const float* po = a.part_o + (base + j) * D + lane;
+#pragma unroll
+            for (int i = 0; i < NC; ++i) xd[j][i] = __ldcg(po + 32 * i);
         }
     }
+    if (E <= 0) return;
+    const int nd = E - 1;  // deep segments with keys
+    float M = mw.x;
+    for (int j = 0; j < nd; ++j) {
+        float2 mj = md[0];
+#pragma unroll
+        for (int q = 1; q < NS0; ++q) mj = j == q ? md[q] : mj;
+        if (j >= NS0) mj = __ldcg(a.part_ml + base + j);
+        M = fmaxf(M, mj.x);
+    }
     float L = 0.f;
-    constexpr int NC = D / 32;
     float acc[NC];
 #pragma unroll
     for (int i = 0; i < NC; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int sg = 0; sg < 9; ++sg) {
-        if (sg < E) {
-            const float f = sm100::ex2(ml[sg].x - M);
-            L = fmaf(ml[sg].y, f, L);
-            const float* po = a.part_o + (base + (sg < E - 1 ? sg : a.nsplit)) * D + lane;
+    for (int j = 0; j < NS0; ++j) {
+        if (j < nd) {
+            const float f = sm100::ex2(md[j].x - M);
+            L = fmaf(md[j].y, f, L);
 #pragma unroll
-            for (int i = 0; i < NC; ++i) acc[i] = fmaf(__ldcg(po + 32 * i), f, acc[i]);
+            for (int i = 0; i < NC; ++i) acc[i] = fmaf(xd[j][i], f, acc[i]);
         }
+    }
+    for (int j = NS0; j < nd; ++j) {  // more than NS0 deep segments (rare)
+        const float2 mj = __ldcg(a.part_ml + base + j);
+        const float* po = a.part_o + (base + j) * D + lane;
+        const float f = sm100::ex2(mj.x - M);
+        L = fmaf(mj.y, f, L);
+#pragma unroll
+        for (int i = 0; i < NC; ++i) acc[i] = fmaf(__ldcg(po + 32 * i), f, acc[i]);
+    }
+    {
+        const float f = sm100::ex2(mw.x - M);
+        L = fmaf(mw.y, f, L);
+#pragma unroll
+        for (int i = 0; i < NC; ++i) acc[i] = fmaf(xw[i], f, acc[i]);
     }
     const float inv = 1.f / L;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.O) + ((int64_t)row * H + h) * D + lane;
@@ -1273,10 +1297,10 @@ __global__ void __launch_bounds__(256) persist_merge_kernel(VerifyArgs a, int nr
 
 template <int D>
 cudaError_t launch_merge(const VerifyArgs& a, int nrows, cudaStream_t st) {
-    const int64_t warps = (int64_t)nrows * a.s.H;
+    const int64_t blocks = ((int64_t)nrows * a.s.H + 3) / 4;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((warps + 7) / 8));
-    cfg.blockDim = dim3(256);
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(128);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1322,10 +1346,9 @@ cudaError_t launch_p(const PMaps& tm, const VerifyArgs& a, const PArgs& pa, int 
 static int persist_kc(int d, int mt) { return d == 128 && mt == 2 ? 48 : 80; }
 
 // Whether the window units run through the stage ring: every unit one chunk (the
-// whole window, the draft tokens) with 8 key rows left for its queries, no sliding
-// window (whose units read more keys).
+// whole window, the draft tokens), no sliding window (whose units read more keys).
 bool persist_ring_ok(int d, int mt, int Wcap, int k, int sliding, int full_box) {
-    return !sliding && full_box && Wcap + k <= persist_kc(d, mt) - 8;
+    return !sliding && full_box && Wcap + k <= persist_kc(d, mt);
 }
 
 // Window warps a CTA of each role runs, for the planner's cost model.

@@ -499,7 +499,7 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
     p.win_ub = (len_ub < c->Wcap ? len_ub : c->Wcap) + max_ntok;
     p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
     if (p.fused && all_depths && plan_persist(c, nbranch / c->R, max_ntok, len_ub, p)) {
-        p.part_bytes = verify_work_bytes(nrows, c->H, c->d, p.nsplit + 1);
+        p.part_bytes = persist_work_bytes(nrows, c->H, c->d, p.nsplit + 1, nbranch / c->R);
         p.work_bytes = p.part_bytes;
         return p;
     }
@@ -554,6 +554,7 @@ cudaError_t launch_verify(const ripe_cache_s* c, const VerifyPlan& plan, int lay
     char* wb = reinterpret_cast<char*>(work);
     a.part_ml = reinterpret_cast<float2*>(wb);
     a.part_o = reinterpret_cast<float*>(wb + verify_ml_bytes(ba.nrows, c->H, a.nseg));
+    a.gE = plan.persist ? reinterpret_cast<int32_t*>(wb + verify_work_bytes(ba.nrows, c->H, c->d, a.nseg)) : nullptr;
     cudaError_t e;
     const int win_ub = plan.win_ub;
     if (plan.persist) {

@@ -17,6 +17,7 @@ struct VerifyArgs {
     float2* part_ml;          // [nrows][H][nseg] (m in log2 units, l)
     float* part_o;            // [nrows][H][nseg][d]
     int q_tma;                // fused kernel: a tensor map of Q came with the launch
+    int32_t* gE;              // persistent kernel: per sequence group, its segment count (0: invalid group)
 };
 
 // Deep splits that hold keys for a sequence whose deep region has A keys.
@@ -31,4 +32,8 @@ inline size_t verify_ml_bytes(int nrows, int H, int nseg) {
 }
 inline size_t verify_work_bytes(int nrows, int H, int d, int nseg) {
     return verify_ml_bytes(nrows, H, nseg) + (size_t)nrows * H * nseg * d * sizeof(float);
+}
+// The persistent kernel's scratch: the partials, then one segment count per group.
+inline size_t persist_work_bytes(int nrows, int H, int d, int nseg, int ngroups) {
+    return verify_work_bytes(nrows, H, d, nseg) + ((size_t)ngroups * sizeof(int32_t) + 255) / 256 * 256;
 }
