@@ -151,7 +151,7 @@ int verify_common(ripe_cache_s* c, int layer, const BranchArgs& ba, const void* 
     if (scale == 0.f) scale = 1.0f / sqrtf((float)c->d);
     // A captured launch replays while the sequences grow: its plan covers Tmax.
     const VerifyPlan plan = plan_verify(c, ba.nbranch, ba.nrows, ba.max_ntok, ba.table == nullptr,
-                                        stream_capturing(st));
+                                        stream_capturing(st), ba.sliding != 0);
     if (ba.sliding && !plan.persist)
         return fail(RIPE_ERR_UNSUPPORTED, "the sliding window needs the persistent sm_100a kernel (bf16, d in "
                     "{64,96,128}, k*R <= 256)");
@@ -442,6 +442,15 @@ int ripe_debug_stall_next_verify(ripe_cache_t c, long long cycles) {
     if (rc != RIPE_OK) return rc;
     if (cycles < 0 || cycles > (1ll << 31)) return fail(RIPE_ERR_INVALID_ARG, "cycles=%lld outside [0, 2^31]", cycles);
     c->probe_cycles.store(cycles);
+    return RIPE_OK;
+}
+
+int ripe_cache_set_all_depths_kernel(ripe_cache_t c, int kernel) {
+    int rc = check_cache(c);
+    if (rc != RIPE_OK) return rc;
+    if (kernel != RIPE_ALL_DEPTHS_AUTO && kernel != RIPE_ALL_DEPTHS_PERSISTENT && kernel != RIPE_ALL_DEPTHS_CLUSTER)
+        return fail(RIPE_ERR_INVALID_ARG, "kernel=%d is not a RIPE_ALL_DEPTHS_* value", kernel);
+    c->all_depths_kernel = kernel;
     return RIPE_OK;
 }
 

@@ -37,6 +37,7 @@ struct ripe_cache_s {
     // Test hook (ripe_debug_stall_next_verify): clock cycles of a wait that nothing
     // ends, taken by the next persistent-kernel verify; 0 = off.
     std::atomic<long long> probe_cycles{0};
+    int all_depths_kernel = 0;  // RIPE_ALL_DEPTHS_* (ripe_cache_set_all_depths_kernel)
 };
 
 // Store geometry, passed by value to kernels.

@@ -41,7 +41,7 @@ struct VerifyPlan {
 // bound on the current lengths -- for launches captured into a CUDA graph, which
 // replay while the sequences grow.
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
-                       bool capacity);
+                       bool capacity, bool sliding = false);
 // True while `st` is being captured into a CUDA graph.
 bool stream_capturing(cudaStream_t st);
 // Re-plan with `nsplit` deep splits (chunk and scratch size follow).

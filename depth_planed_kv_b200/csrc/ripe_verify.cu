@@ -488,7 +488,7 @@ int device_sm_count() {
 }
 
 VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_ntok, bool all_depths,
-                       bool capacity) {
+                       bool capacity, bool sliding) {
     VerifyPlan p{};
     p.max_ntok = max_ntok;
     p.nrowchunks = (max_ntok + kRowsPerCta - 1) / kRowsPerCta;
@@ -498,7 +498,17 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
     p.a_ub = A_ub;
     p.win_ub = (len_ub < c->Wcap ? len_ub : c->Wcap) + max_ntok;
     p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
-    if (p.fused && all_depths && plan_persist(c, nbranch / c->R, max_ntok, len_ub, p)) {
+    // All depths: the persistent kernel for the sliding window (only it serves that
+    // form) and where the deep region outweighs the windows over enough (sequence,
+    // head) pairs to fill the SMs -- long contexts; measured on B200, the cluster
+    // kernel is as fast or faster for short contexts and wide windows.
+    const int nseq = all_depths ? nbranch / c->R : 0;
+    const int deep_ub = len_ub > c->W ? len_ub - c->W : 0;
+    const bool deep_heavy = (int64_t)deep_ub >= (int64_t)c->R * (c->Wcap + max_ntok) &&
+                            (int64_t)nseq * c->H >= device_sm_count();
+    const int choice = c->all_depths_kernel;
+    const bool want = sliding || choice == RIPE_ALL_DEPTHS_PERSISTENT || (choice == RIPE_ALL_DEPTHS_AUTO && deep_heavy);
+    if (p.fused && all_depths && want && plan_persist(c, nseq, max_ntok, len_ub, p)) {
         p.part_bytes = persist_work_bytes(nrows, c->H, c->d, p.nsplit + 1, nbranch / c->R);
         p.work_bytes = p.part_bytes;
         return p;

@@ -73,6 +73,7 @@ _sig("ripe_verify_attn_noalloc", [_P, _I, _P, _I, _I, _P, _P, _P, _P, ctypes.c_f
 _sig("ripe_reserve_workspace", [_P, _I])
 _sig("ripe_synth_fill", [_P, _P, _P, _I, ctypes.c_uint64, _P, _P])
 _sig("ripe_cache_verify_path", [_P, ctypes.POINTER(_I)])
+_sig("ripe_cache_set_all_depths_kernel", [_P, _I])
 _sig("ripe_debug_stall_next_verify", [_P, ctypes.c_longlong])
 _sig("ripe_accept", [_I, _I, _I, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P])
 _sig("ripe_cache_buffers", [_P] + [ctypes.POINTER(_P)] * 7)
@@ -85,7 +86,8 @@ _sig("ripe_last_error", [], ctypes.c_char_p)
 EXPORTED = ["ripe_cache_bytes", "ripe_cache_create", "ripe_cache_destroy", "ripe_cache_reset",
             "ripe_append", "ripe_evict", "ripe_truncate", "ripe_fork", "ripe_read_forks", "ripe_verify_attn",
             "ripe_verify_attn_all_depths", "ripe_verify_attn_all_depths_sliding", "ripe_verify_attn_noalloc", "ripe_reserve_workspace",
-            "ripe_synth_fill", "ripe_cache_verify_path", "ripe_debug_stall_next_verify", "ripe_accept",
+            "ripe_synth_fill", "ripe_cache_verify_path", "ripe_cache_set_all_depths_kernel",
+            "ripe_debug_stall_next_verify", "ripe_accept",
             "ripe_cache_buffers", "ripe_read_meta", "ripe_get_device_error", "ripe_launch_count",
             "ripe_error_string", "ripe_last_error"]
 
@@ -273,6 +275,13 @@ class RipeCache:
         """Test hook: the next persistent-kernel verify waits `cycles` on a barrier
         nothing signals, so its bounded wait runs out (RIPE_DEVERR_TIMEOUT)."""
         _check(_lib.ripe_debug_stall_next_verify(self.handle, int(cycles)), "ripe_debug_stall_next_verify")
+
+    ALL_DEPTHS_AUTO, ALL_DEPTHS_PERSISTENT, ALL_DEPTHS_CLUSTER = 0, 1, 2
+
+    def ripe_cache_set_all_depths_kernel(self, kernel: int):
+        """Which sm_100a kernel serves the all-depths verify (0 auto, 1 persistent,
+        2 cluster); the sliding form always runs in the persistent kernel."""
+        _check(_lib.ripe_cache_set_all_depths_kernel(self.handle, int(kernel)), "ripe_cache_set_all_depths_kernel")
 
     def ripe_cache_verify_path(self) -> int:
         """1: the fused sm_100a kernel serves verify; 0: the CUDA-core kernels."""

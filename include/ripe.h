@@ -316,6 +316,22 @@ enum { RIPE_PATH_CUDA_CORE = 0, RIPE_PATH_FUSED_SM100 = 1 };
 int ripe_cache_verify_path(ripe_cache_t cache, int* path);
 
 /*
+ * Which sm_100a kernel serves ripe_verify_attn_all_depths on this cache (a
+ * scheduling choice; both compute the same rows, and the pages have no
+ * counterpart):
+ *   RIPE_ALL_DEPTHS_AUTO (0, the default): the persistent kernel where the deep
+ *     region outweighs the windows (deep length >= R * (Wcap + k)) over at least
+ *     as many (sequence, head) pairs as the GPU has SMs, else the cluster kernel;
+ *   RIPE_ALL_DEPTHS_PERSISTENT (1): the persistent kernel whenever it can serve
+ *     the call (k*R <= 256);
+ *   RIPE_ALL_DEPTHS_CLUSTER (2): the cluster kernel.
+ * The sliding form always runs in the persistent kernel.  RIPE_ERR_INVALID_ARG
+ * for another value; the setting takes effect from the next call.
+ */
+enum { RIPE_ALL_DEPTHS_AUTO = 0, RIPE_ALL_DEPTHS_PERSISTENT = 1, RIPE_ALL_DEPTHS_CLUSTER = 2 };
+int ripe_cache_set_all_depths_kernel(ripe_cache_t cache, int kernel);
+
+/*
  * The acceptance step of self-speculative decoding, in LoopSpec's order (LoopSpec
  * article, sections on the second branch and on the final check): for each draft
  * position, first the early draft x1 is tested against the final distribution,

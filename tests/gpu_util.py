@@ -18,10 +18,15 @@ def torch_dtype(wl):
     return torch.bfloat16 if wl.bf16 else torch.float32
 
 
-def make_cache(wl, nseq=None, Tmax=None):
+def make_cache(wl, nseq=None, Tmax=None, kernel=0):
+    """kernel: which sm_100a kernel serves all-depths calls (0 auto, 1 persistent,
+    2 cluster)."""
     from depth_planed_kv_b200.ripe import RipeCache
-    return RipeCache(wl.layers, wl.R, wl.H, wl.d, wl.W, Tmax or wl.Tmax, nseq or wl.nseq, wl.kmax,
-                     torch_dtype(wl))
+    cache = RipeCache(wl.layers, wl.R, wl.H, wl.d, wl.W, Tmax or wl.Tmax, nseq or wl.nseq, wl.kmax,
+                      torch_dtype(wl))
+    if kernel:
+        cache.ripe_cache_set_all_depths_kernel(kernel)
+    return cache
 
 
 def fill(cache, wl, ctx):

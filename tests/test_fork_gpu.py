@@ -22,14 +22,17 @@ def _vals(rng, shape, bf16):
     return S.round_bf16(x) if bf16 else x
 
 
-@pytest.mark.parametrize("dtype,d,T0", [(torch.bfloat16, 96, 300), (torch.bfloat16, 64, 130),
-                                        (torch.float32, 16, 200)])
-def test_verify_on_a_fork_matches_oracle(dtype, d, T0):
+@pytest.mark.parametrize("dtype,d,T0,kernel", [(torch.bfloat16, 96, 300, 1), (torch.bfloat16, 96, 300, 2),
+                                               (torch.bfloat16, 64, 130, 1), (torch.bfloat16, 64, 130, 2),
+                                               (torch.float32, 16, 200, 0)])
+def test_verify_on_a_fork_matches_oracle(dtype, d, T0, kernel):
     from depth_planed_kv_b200.ripe import RipeCache, branch_table
     bf16 = dtype == torch.bfloat16
     L, R, H, W, kmax, Tmax, B = 1, 4, 2, 16, 4, 400, 4
     wl = S.Workload("fork", L, R, H, d, W, kmax, B, None, 0.88, 0, "bf16" if bf16 else "f32", Tmax, kmax)
     cache = RipeCache(L, R, H, d, W, Tmax, B, kmax, dtype)
+    if kernel:
+        cache.ripe_cache_set_all_depths_kernel(kernel)   # 1 persistent, 2 cluster
     model = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np.float32)
     rng = np.random.default_rng(d + T0)
     dev = lambda a: torch.from_numpy(np.asarray(a, np.int32)).cuda()

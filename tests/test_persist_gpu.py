@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _verify_and_check(wl, ctx, heads=None, ctx_len=None, reps=1):
-    cache = make_cache(wl, nseq=len(ctx))
+    cache = make_cache(wl, nseq=len(ctx), kernel=1)
     assert cache.ripe_cache_verify_path() == 1
     fill(cache, wl, ctx)
     nseq = len(ctx)

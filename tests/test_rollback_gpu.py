@@ -20,17 +20,19 @@ def _vals(rng, shape, bf16):
     return S.round_bf16(x) if bf16 else x
 
 
+@pytest.mark.parametrize("kernel", [1, 2])   # all-depths calls: persistent / cluster kernel
 @pytest.mark.parametrize("dtype,d,W,kmax", [
-    (torch.bfloat16, 64, 16, 4),   # fused sm_100a kernel, W >= block
-    (torch.bfloat16, 128, 3, 8),   # fused kernel, W < block
+    (torch.bfloat16, 64, 16, 4),   # fused sm_100a kernels, W >= block
+    (torch.bfloat16, 128, 3, 8),   # fused kernels, W < block
     (torch.float32, 16, 5, 4),     # CUDA-core kernels
 ])
-def test_verify_after_rollback_matches_oracle(dtype, d, W, kmax):
+def test_verify_after_rollback_matches_oracle(dtype, d, W, kmax, kernel):
     from depth_planed_kv_b200.ripe import RipeCache
     bf16 = dtype == torch.bfloat16
     wl = S.Workload("rollback", 1, 4, 2, d, W, kmax, 2, None, 0.88, 0, "bf16" if bf16 else "f32", 256, kmax)
     L, R, H, B, Tmax = 1, wl.R, wl.H, 2, wl.Tmax
     cache = RipeCache(L, R, H, d, W, Tmax, B, kmax, dtype)
+    cache.ripe_cache_set_all_depths_kernel(kernel)
     model = OR.OracleStore(L, R, H, d, W, Tmax, B, kmax, np.float32)
     rng = np.random.default_rng(7 + d + W)
     ids = np.array([0, 1], np.int32)

@@ -17,7 +17,7 @@ def test_expired_wait_reports_timeout_and_next_call_is_exact():
     from depth_planed_kv_b200.ripe import RIPE_OK
     wl = S.Workload("timeout", 1, 4, 3, 64, 16, 4, 2, None, 0.88, 1301, "bf16", 600, 4)
     ctx = np.array([500, 130])
-    cache = make_cache(wl)
+    cache = make_cache(wl, kernel=1)   # the hook stalls the persistent kernel
     assert cache.ripe_cache_verify_path() == 1
     fill(cache, wl, ctx)
     ws = [int(t) - wl.W for t in ctx]

@@ -99,11 +99,12 @@ def test_huginn_rows_ignore_other_depths_and_later_tokens(huginn_cache):
 
 # --- window sweep at the Huginn shape ---------------------------------------------
 
+@pytest.mark.parametrize("kernel", [1, 2])   # persistent / cluster kernel
 @pytest.mark.parametrize("W", S.SWEEP_W)
-def test_window_sweep(W):
+def test_window_sweep(W, kernel):
     wl = S.sweep(W)
     wl.layers = 1
-    cache = make_cache(wl)
+    cache = make_cache(wl, kernel=kernel)
     fill(cache, wl, [wl.ctx])
     _, O, lse, _ = run_all_depths(cache, wl, 0, 1, wl.k)
     heads = np.array([0, 9, 31, 54])
