@@ -422,14 +422,15 @@ def make_mixed_work(rank):
     return wk
 
 
-def make_long_work(rank, peaks):
+def make_long_work(rank, peaks, small=False):
     """Long context: verify all depths of 16 sequences at T=32768, then append U[1,8]
     accepted tokens per sequence (their planes are the verified block's) and evict;
-    16 timed steps, the contexts grow."""
+    16 timed steps, the contexts grow.  `small`: 6 sequences at T=8192, the case
+    the profiler captures."""
     import torch
-    from depth_planed_kv_b200.ripe import RipeCache
+    from depth_planed_kv_b200.ripe import RipeCache, ripe_cache_bytes
     from depth_planed_kv_b200.synth_rows import all_depth_rows
-    wl = S.long_context()
+    wl = S.long_context_small() if small else S.long_context()
     B, R, H, d, k = wl.nseq, wl.R, wl.H, wl.d, wl.k
     cache = RipeCache(1, R, H, d, wl.W, wl.Tmax, B, wl.kmax, torch.bfloat16)
     cache.ripe_synth_fill(list(range(B)), [wl.ctx] * B, shard_seed(wl.seed, rank), S.coef_table(wl.decay, R))
@@ -444,10 +445,12 @@ def make_long_work(rank, peaks):
     for i in range(64):
         T = T + n_acc[i]
         lens.append(T.copy())
-    wk = Work("long_ctx", {"workload": "long_ctx_B16_T32768", "layers": 1, "R": R, "H": H, "d": d, "T": wl.ctx,
+    wk = Work("long_ctx", {"workload": wl.name, "layers": 1, "R": R, "H": H, "d": d, "T": wl.ctx,
                            "W": wl.W, "k": k, "sequences": B,
                            "step": "verify all depths + append U[1,8] accepted tokens + evict; contexts grow",
-                           "l2": "inputs larger than L2: 10 GB store"}, cache, 1, 1)
+                           "l2": "inputs larger than L2: %.1f GB store" %
+                                 (ripe_cache_bytes(1, R, H, d, wl.W, wl.Tmax, B, wl.kmax, torch.bfloat16) / 1e9)},
+              cache, 1, 1)
     pairs = [pinned_pair(x.reshape(shape), torch.bfloat16) for x in (Q, Kb, Vb)]
     nacc_h, nacc_d = pinned_pair(n_acc, torch.int32)
     wk.host_in = [[[p[0] for p in pairs] + [nacc_h]]]
@@ -670,6 +673,8 @@ def build_work(name, rank, peaks):
         return make_mixed_work(rank)
     if name == "long_ctx":
         return make_long_work(rank, peaks)
+    if name == "long_ctx_small":
+        return make_long_work(rank, peaks, small=True)
     raise ValueError(name)
 
 
@@ -713,7 +718,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ripe", choices=["ripe", "reference"])
-    ap.add_argument("--workload", default="huginn", choices=WORKLOADS + ["all"])
+    ap.add_argument("--workload", default="huginn", choices=WORKLOADS + ["all", "long_ctx_small"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -186,6 +186,13 @@ def long_context() -> Workload:
                     32768 + 512, 8)
 
 
+def long_context_small() -> Workload:
+    """The long-context step at 6 sequences x 8192 (about 2.2 GB of store): a
+    case small enough for a full profiler capture of the same kernels."""
+    return Workload("long_ctx_B6_T8192", 1, 32, 32, 128, 128, 8, 6, 8192, 0.88, 1005, "bf16",
+                    8192 + 512, 8)
+
+
 @dataclasses.dataclass
 class BranchSpec:
     seq: int
