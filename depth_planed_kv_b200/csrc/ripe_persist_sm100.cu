@@ -95,29 +95,38 @@ struct PLayout {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + ST * KV_STAGE;
     static constexpr int OFF_W = OFF_V + ST * KV_STAGE;
-    static constexpr int OFF_WEND = OFF_W + NWW * WSTAGE;
     static constexpr int THREADS = 32 * (kDeepWarps + NWW);
     static constexpr int NWARPS = THREADS / 32;
-    // A CTA without deep items: window stages over the whole stage region.
-    static constexpr int NW_FULL = (OFF_WEND / WSTAGE) < NWARPS ? (OFF_WEND / WSTAGE) : NWARPS;
-    static constexpr int OFF_OST = OFF_WEND;  // epilogue staging of the softmax warps
     static constexpr int OST_BYTES = 4 * 8 * (32 * 4 + 16);
-    static constexpr int OFF_BAR = OFF_OST + OST_BYTES;
     // q_full, k_full[ST], v_full[ST], kv_empty[ST], s_full[2], p_full[2], pv_done[2], drain, epi_done, probe
     static constexpr int NBAR = 1 + 3 * ST + 9;
+    static constexpr int DESC_BYTES = 96;
+    static constexpr int ITEM_BYTES = (kMaxItems * (int)sizeof(DeepItem) + 15) / 16 * 16;
+    // What follows the stage region: softmax staging, barriers, flags, tables.
+    static constexpr int TAIL = OST_BYTES + NBAR * 8 + 2 * NWARPS * 8 + 64 + ITEM_BYTES + NWARPS * DESC_BYTES +
+                                NWARPS * 4 + NWARPS + 64;
+    static constexpr int SMEM_CAP = 232448;  // 227 KB per CTA
+    // The stage region takes the rest of the budget: the deep stages, then window
+    // stages of a deep CTA; a CTA without deep items puts window stages everywhere.
+    static constexpr int OFF_WEND = (SMEM_CAP - 1024 - TAIL) / 1024 * 1024;
+    static constexpr int NS_DEEP_RAW = (OFF_WEND - OFF_W) / WSTAGE;
+    static constexpr int NS_DEEP = NS_DEEP_RAW < NWARPS ? NS_DEEP_RAW : NWARPS;  // window stages of a deep CTA
+    static constexpr int NW_FULL = (OFF_WEND / WSTAGE) < NWARPS ? (OFF_WEND / WSTAGE) : NWARPS;
+    static constexpr int OFF_OST = OFF_WEND;  // epilogue staging of the softmax warps
+    static constexpr int OFF_BAR = OFF_OST + OST_BYTES;
     // Window stage barriers: one per warp (full), then one per warp (empty, stage ring).
     static constexpr int OFF_WBAR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_MISC = OFF_WBAR + 2 * NWARPS * 8;
     static constexpr int OFF_ITEMS = OFF_MISC + 64;
     // Stage ring: the unit held by each stage.
-    static constexpr int DESC_BYTES = 96;
-    static constexpr int OFF_DESC = (OFF_ITEMS + kMaxItems * (int)sizeof(DeepItem) + 15) / 16 * 16;
+    static constexpr int OFF_DESC = OFF_ITEMS + ITEM_BYTES;
     // Stage ring: the ticket last issued into each stage.
     static constexpr int OFF_ISS = OFF_DESC + NWARPS * DESC_BYTES;
     // Stage ring: whether a stage's last use wrote window rows by 16-byte copies.
     static constexpr int OFF_DIRTY = OFF_ISS + NWARPS * 4;
     static constexpr int BYTES = OFF_DIRTY + NWARPS;
     static constexpr int SMEM = BYTES + 1024;
+    static_assert(NS_DEEP >= 1, "a deep CTA needs a window stage");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL(int mt, int sb) { return (uint32_t)((mt * 2 + sb) * kN); }
     static constexpr uint32_t O_COL(int mt) { return (uint32_t)(MT * 2 * kN + mt * 128); }
@@ -1022,7 +1031,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             // ---- stage ring: full[st] (33 arrivals: 32 lanes' copies + the expect_tx),
             // empty[st] (the consumer that read it), the unit in desc[st].
             static_assert(sizeof(Unit) <= Lay::DESC_BYTES, "unit descriptor");
-            const int NS = deep_cta ? NWW : Lay::NW_FULL;
+            const int NS = deep_cta ? Lay::NS_DEEP : Lay::NW_FULL;
             uint8_t* sring = sm + (deep_cta ? Lay::OFF_W : 0);
             uint64_t* full = wbar;
             uint64_t* empty = wbar + Lay::NWARPS;
@@ -1203,7 +1212,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     if (RING && threadIdx.x == 0 && *abort_flag) {
         // A ring that gave up may still have tensor copies in flight: wait for the
         // last phase issued into each stage before the shared memory goes away.
-        const int NS = deep_cta ? NWW : Lay::NW_FULL;
+        const int NS = deep_cta ? Lay::NS_DEEP : Lay::NW_FULL;
         const int* iss = reinterpret_cast<const int*>(sm + Lay::OFF_ISS);
         volatile int no_abort = 0;
         for (int st = 0; st < NS; ++st)
@@ -1316,6 +1325,8 @@ template <int D, int MT, int ST, int NWW, int KC, bool RING>
 cudaError_t launch_p(const PMaps& tm, const VerifyArgs& a, const PArgs& pa, int grid, cudaStream_t st) {
     using Lay = PLayout<D, MT, ST, NWW, KC>;
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
+    // Per-warp stages: every window warp of a deep CTA owns a stage.
+    static_assert(RING || Lay::NS_DEEP >= NWW, "window stages of a deep CTA");
     static PerDeviceOnce configured;
     cudaError_t ce = per_device_once(configured, [] {
         cudaError_t e = cudaFuncSetAttribute(persist_kernel<D, MT, ST, NWW, KC, RING>,
@@ -1395,19 +1406,22 @@ cudaError_t launch_persist(const void* tmaps, const VerifyArgs& args, int pd, in
     const bool ring = persist_ring_ok(d, mt, a.s.Wcap, a.ba.k, sliding, full_box);
     // The kernel publishes every partial; the merge kernel (its dependent launch)
     // combines them.
-#define RIPE_LAUNCH(D_, MT_, ST_, NWW_, KC_)                                                 \
-    if (d == D_ && mt == MT_) {                                                           \
-        cudaError_t e = ring ? launch_p<D_, MT_, ST_, NWW_, KC_, true>(tm, a, pa, grid, st)  \
-                             : launch_p<D_, MT_, ST_, NWW_, KC_, false>(tm, a, pa, grid, st); \
-        if (e != cudaSuccess) return e;                                                   \
-        return launch_merge<D_>(a, a.ba.nrows, st);                                       \
+    // Deep stages: ST_ with per-warp window stages; STR_ with the ring, whose deep
+    // CTAs need only a stage or two for their few window units (the deep pipeline is
+    // bound by its bytes in flight).
+#define RIPE_LAUNCH(D_, MT_, ST_, STR_, NWW_, KC_)                                            \
+    if (d == D_ && mt == MT_) {                                                            \
+        cudaError_t e = ring ? launch_p<D_, MT_, STR_, NWW_, KC_, true>(tm, a, pa, grid, st)  \
+                             : launch_p<D_, MT_, ST_, NWW_, KC_, false>(tm, a, pa, grid, st);  \
+        if (e != cudaSuccess) return e;                                                    \
+        return launch_merge<D_>(a, a.ba.nrows, st);                                        \
     }
-    RIPE_LAUNCH(64, 1, 4, 6, 80)
-    RIPE_LAUNCH(96, 1, 4, 4, 80)
-    RIPE_LAUNCH(128, 1, 3, 3, 80)
-    RIPE_LAUNCH(64, 2, 4, 5, 80)
-    RIPE_LAUNCH(96, 2, 3, 3, 80)
-    RIPE_LAUNCH(128, 2, 3, 2, 48)
+    RIPE_LAUNCH(64, 1, 4, 8, 6, 80)
+    RIPE_LAUNCH(96, 1, 4, 6, 4, 80)
+    RIPE_LAUNCH(128, 1, 3, 4, 3, 80)
+    RIPE_LAUNCH(64, 2, 4, 4, 5, 80)
+    RIPE_LAUNCH(96, 2, 3, 3, 3, 80)
+    RIPE_LAUNCH(128, 2, 3, 3, 2, 48)
 #undef RIPE_LAUNCH
     return cudaErrorInvalidValue;
 }
