@@ -144,8 +144,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Context of sequence slot g of an all-depths call: its id, committed length T,
-// deep-region length A and the arrivals E each of its slices expects; ok is
-// false for an id outside the store (reported once).
+// deep-region length A and the number E of partial segments of each of its rows
+// (deep chunks with keys, plus the window); ok is false for an id outside the
+// store (reported once).
 struct GroupCtx {
     int seq, T, A, E, fb, fp;  // fb, fp: deep positions below fp are read from sequence fb
     bool ok;
@@ -609,19 +610,16 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
     // with a stage anywhere in the stage region.  Warps take the CTA's units one at
     // a time from a shared counter.  Each runs a unit one chunk of keys at a time
     // through its own stage; when a unit's last chunk has been read out of the
-    // stage, the warp issues the next unit's first chunk and its Q loads, publishes
-    // the unit's partial and arrives, and looks at whether that arrival was the last
-    // only when the next unit ends (with the unit after it in flight), so that the
-    // round trips overlap.
-    // Stage ring (every unit one chunk, its queries in the chunk's last 8 key rows):
-    // one producer warp (the first window warp) walks the CTA's units in order and
-    // loads each into the next free stage of a ring; every other warp (the deep
-    // warps too, once their items are done) is a consumer that takes the next
-    // ticket, waits for that stage, computes, frees the stage at once and only then
-    // publishes and arrives.  The loads run ahead of the arrivals' round trips.
+    // stage, the warp issues the next unit's first chunk and its Q loads, then
+    // publishes the unit's partial.
+    // Stage ring (every unit one chunk): producer warps (the first window warps)
+    // walk the CTA's units in order and load each into the next free stage of a
+    // ring; every other warp (the deep warps too, once their items are done) is a
+    // consumer that takes the next ticket, waits for that stage, computes, frees the
+    // stage at once and only then publishes.
     constexpr int NX = Lay::OFF_W / Lay::WSTAGE < kDeepWarps ? Lay::OFF_W / Lay::WSTAGE : kDeepWarps;
     if (deep_cta && warp < kDeepWarps) asm volatile("bar.sync 2, %0;" ::"n"(32 * kDeepWarps) : "memory");
-    const int wfirst = deep_cta ? kDeepWarps : 0;  // the ring's producer
+    const int wfirst = deep_cta ? kDeepWarps : 0;  // the ring's first producer
     const bool win_role = RING ? true : deep_cta ? (warp >= kDeepWarps || warp < NX) : warp < Lay::NW_FULL;
     if (win_role) {
         uint8_t* stage = sm + (deep_cta && warp >= kDeepWarps ? Lay::OFF_W + (warp - kDeepWarps) * Lay::WSTAGE
@@ -659,7 +657,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             int g, h, r, j0, nr, nw, nblk, ndw, nbr, nk, koff, slot0, sbase, E, A, seq, fb, fp;
             bool ring, slide, ok, fast;
         };
-        // What the merge of a unit's slice needs.
+        // The rows a unit's partial belongs to.
         struct Slice {
             int g, h, r, j0, nr, E;
         };
