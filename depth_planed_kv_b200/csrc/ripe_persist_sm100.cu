@@ -994,6 +994,94 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
             __syncwarp();  // every lane is done reading the stage
         };
 
+        // A whole unit (every key in the stage, no sliding window) in one pass: S^T of
+        // all its 16-key tiles (independent accumulation chains), the visibility mask,
+        // one row max, the probabilities and O^T = V^T P^T.  The unit's keys fit in
+        // registers, so no running rescale is needed; the chain from the stage's
+        // arrival to its release is a few hundred cycles.
+        auto compute_whole = [&](const Unit& w, uint32_t sb_in, const uint32_t (&bq)[NKS][2], float (&o)[NMT][4],
+                                 float& m_a, float& m_b, float& l_a, float& l_b) {
+            const int nt = (w.nk + 15) / 16;  // <= NT (the producer checked nk <= KC)
+            const uint32_t sb = smem_ready(sb_in);
+            float sc[NT][4];
+#pragma unroll
+            for (int u = 0; u < NT; ++u) {
+                sc[u][0] = sc[u][1] = sc[u][2] = sc[u][3] = 0.f;
+                if (u < nt) {
+#pragma unroll
+                    for (int ks = 0; ks < NKS; ++ks) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_r(sb + (ks >> 1) * Lay::KCB + (16 * u + rk) * 64 + ((ks & 1) ? k_sw1 : k_sw0), a0, a1,
+                                  a2, a3);
+                        mma_16816(sc[u], a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+                    }
+                }
+            }
+            // Key kk is visible to row j if it is a live window slot (whole-window ring
+            // units: slot kk holds position A + ((kk - A) mod Wcap)), or draft token
+            // kk - koff <= j.  Keys past the unit's are draft indices >= nblk.
+            const bool wrap = w.fast && w.ring;
+            float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < NT; ++u) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int kk = 16 * u + r8 + 8 * hf;
+                    bool va, vb;
+                    if (kk < w.koff) {
+                        int i = kk;
+                        if (wrap) {
+                            i += s.Wcap - w.slot0;
+                            if (i >= s.Wcap) i -= s.Wcap;
+                        }
+                        va = vb = i < w.nw;
+                    } else {
+                        const int e = kk - w.koff;
+                        va = e < w.nblk && e <= w.j0 + ra;
+                        vb = e < w.nblk && e <= w.j0 + rb;
+                    }
+                    float& xa = sc[u][2 * hf];
+                    float& xb = sc[u][2 * hf + 1];
+                    xa = va ? xa * c2 : -INFINITY;
+                    xb = vb ? xb * c2 : -INFINITY;
+                    mx_a = fmaxf(mx_a, xa);
+                    mx_b = fmaxf(mx_b, xb);
+                }
+            }
+#pragma unroll
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, o2));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, o2));
+            }
+            m_a = mx_a;
+            m_b = mx_b;
+            float la = 0.f, lb = 0.f;
+#pragma unroll
+            for (int u = 0; u < NT; ++u) {
+                if (u < nt) {
+                    const float p0 = mx_a == -INFINITY ? 0.f : ex2(sc[u][0] - mx_a);
+                    const float p1 = mx_b == -INFINITY ? 0.f : ex2(sc[u][1] - mx_b);
+                    const float p2 = mx_a == -INFINITY ? 0.f : ex2(sc[u][2] - mx_a);
+                    const float p3 = mx_b == -INFINITY ? 0.f : ex2(sc[u][3] - mx_b);
+                    la += p0 + p2;
+                    lb += p1 + p3;
+                    const uint32_t pb0 = movmatrix_t(pack_bf16(p0, p1));
+                    const uint32_t pb1 = movmatrix_t(pack_bf16(p2, p3));
+#pragma unroll
+                    for (int mt = 0; mt < NMT; ++mt) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_t_r(sb + NCH * Lay::KCB + (mt >> 1) * Lay::KCB + (16 * u + rv) * 64 +
+                                        ((mt & 1) ? v_sw1 : v_sw0),
+                                    a0, a1, a2, a3);
+                        mma_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+                    }
+                }
+            }
+            l_a = la;
+            l_b = lb;
+            __syncwarp();  // every lane is done reading the stage
+        };
+
         // Publish a unit's partial (segment nsplit of its rows).
         auto publish = [&](const Slice& w, const float (&o)[NMT][4], float m_a, float m_b, float l_a, float l_b) {
 #pragma unroll
@@ -1076,8 +1164,8 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     }
                     Unit w = describe_at(cg, ch, cr, cq);
                     for (int i = 0; i < NP; ++i) step();
-                    // every unit here is one chunk
-                    if (w.ok && w.nk > KC) {
+                    // every unit here is one chunk, without the sliding window
+                    if (w.ok && (w.nk > KC || w.slide)) {
                         if (lane == 0) set_device_error(s.err, RIPE_DEVERR_BRANCH);
                         w.ok = false;
                     }
@@ -1139,7 +1227,7 @@ persist_kernel(const __grid_constant__ PMaps tm, VerifyArgs a, PArgs pa) {
                     if (w.ok) {
 #pragma unroll
                         for (int mt = 0; mt < NMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-                        compute(w, 0, sa, bq, o, m_a, m_b, l_a, l_b);
+                        compute_whole(w, sa, bq, o, m_a, m_b, l_a, l_b);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(empty + st);  // the stage is free again

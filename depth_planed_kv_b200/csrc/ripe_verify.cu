@@ -499,15 +499,21 @@ VerifyPlan plan_verify(const ripe_cache_s* c, int nbranch, int nrows, int max_nt
     p.win_ub = (len_ub < c->Wcap ? len_ub : c->Wcap) + max_ntok;
     p.fused = c->tc_ready && fused_supported(c->dtype, c->d);
     // All depths: the persistent kernel for the sliding window (only it serves that
-    // form) and where the deep region outweighs the windows over enough (sequence,
-    // head) pairs to fill the SMs -- long contexts; measured on B200, the cluster
-    // kernel is as fast or faster for short contexts and wide windows.
+    // form); where the deep region outweighs the windows over enough (sequence, head)
+    // pairs to fill the SMs (long contexts); and where the windows, each one stage of
+    // its ring, outweigh the deep region (short contexts, windows of tens of
+    // positions).  Measured on B200, the cluster kernel is faster for windows too wide
+    // for one stage and for windows of a few positions over a longer deep region.
     const int nseq = all_depths ? nbranch / c->R : 0;
     const int deep_ub = len_ub > c->W ? len_ub - c->W : 0;
     const bool deep_heavy = (int64_t)deep_ub >= (int64_t)c->R * (c->Wcap + max_ntok) &&
                             (int64_t)nseq * c->H >= device_sm_count();
+    const int mt_ad = max_ntok * c->R > 128 ? 2 : 1;
+    const bool window_heavy = persist_ring_ok(c->d, mt_ad, c->Wcap, max_ntok, sliding ? 1 : 0, c->full_box ? 1 : 0) &&
+                              (int64_t)c->R * c->Wcap >= deep_ub;
     const int choice = c->all_depths_kernel;
-    const bool want = sliding || choice == RIPE_ALL_DEPTHS_PERSISTENT || (choice == RIPE_ALL_DEPTHS_AUTO && deep_heavy);
+    const bool want = sliding || choice == RIPE_ALL_DEPTHS_PERSISTENT ||
+                      (choice == RIPE_ALL_DEPTHS_AUTO && (deep_heavy || window_heavy));
     if (p.fused && all_depths && want && plan_persist(c, nseq, max_ntok, len_ub, p)) {
         p.part_bytes = persist_work_bytes(nrows, c->H, c->d, p.nsplit + 1, nbranch / c->R);
         p.work_bytes = p.part_bytes;

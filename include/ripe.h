@@ -321,7 +321,10 @@ int ripe_cache_verify_path(ripe_cache_t cache, int* path);
  * counterpart):
  *   RIPE_ALL_DEPTHS_AUTO (0, the default): the persistent kernel where the deep
  *     region outweighs the windows (deep length >= R * (Wcap + k)) over at least
- *     as many (sequence, head) pairs as the GPU has SMs, else the cluster kernel;
+ *     as many (sequence, head) pairs as the GPU has SMs, or where the windows
+ *     outweigh the deep region (R * Wcap >= deep length) and each window with the
+ *     k draft tokens fits one stage of the kernel's ring (Wcap + k <= 80, or 48
+ *     for d = 128 with k*R > 128), else the cluster kernel;
  *   RIPE_ALL_DEPTHS_PERSISTENT (1): the persistent kernel whenever it can serve
  *     the call (k*R <= 256);
  *   RIPE_ALL_DEPTHS_CLUSTER (2): the cluster kernel.

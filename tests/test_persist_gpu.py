@@ -1,9 +1,9 @@
 """The persistent all-depths kernel against the fp64 oracle: several sequences
-with ragged contexts (deep items and window units spread over the grid, slices
-merged by whichever arrival comes last), one and two 128-row M tiles, slices of
-fewer than eight tokens, contexts inside the window, empty windows, many deep
-items per CTA, the context-length override, and repeated calls (the slice
-counters return to zero, the merge order is fixed)."""
+with ragged contexts (deep items and window units spread over the grid), one and
+two 128-row M tiles, slices of fewer than eight tokens, contexts inside the window,
+empty windows, many deep items per CTA, the context-length override, repeated
+calls (the merge order is fixed), and calls of the cluster kernel and over fewer
+sequences in between (both kernels share the cache's scratch)."""
 import numpy as np
 import pytest
 import torch
@@ -79,3 +79,22 @@ def test_many_window_units_per_cta(W):
     # units on each CTA, so the stage ring's producer warps run far apart.
     wl = S.Workload("p_units_w%d" % W, 1, 32, 55, 96, W, 4, 1, None, 0.88, 1206, "bf16", 1088, 4)
     _verify_and_check(wl, np.array([1024]), heads=[0, 17, 54], reps=2)
+
+
+def test_interleaved_kernels_and_subsets():
+    # Persistent and cluster-kernel calls alternate on one cache (they share its
+    # scratch), over all three sequences or fewer.
+    wl = S.Workload("p_mix", 1, 32, 6, 96, 64, 4, 3, None, 0.88, 1207, "bf16", 1200, 4)
+    cache = make_cache(wl, nseq=3, kernel=1)
+    ctx = np.array([1100, 700, 80])
+    fill(cache, wl, ctx)
+    ws = [max(0, int(t) - wl.W) for t in ctx]
+    ref, ref_lse = oracle_all_depths(wl, 0, 3, wl.k, [int(t) for t in ctx], ws)
+    rows = wl.k * wl.R
+    for kern, n in [(1, 3), (2, 3), (1, 3), (1, 1), (2, 2), (1, 3), (1, 2), (1, 3)]:
+        cache.ripe_cache_set_all_depths_kernel(kern)
+        _, O, lse, _ = run_all_depths(cache, wl, 0, n, wl.k)
+        check(O, ref[: n * rows], wl, "kernel %d, %d sequences" % (kern, n))
+        check_lse(lse, ref_lse[: n * rows])
+    assert cache.ripe_get_device_error() == 0
+    cache.close()
