@@ -568,7 +568,7 @@ def run_work(wk, args, world, rank, local, peaks, peak_kind):
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_for(wk.config["workload"]),
             "peak_source": peak_kind,
-            "kernel": "the verify call: the persistent kernel and its merge kernel (one ripe_verify_attn* call); CUDA events on their stream"}
+            "kernel": "the verify call (one ripe_verify_attn* call: the persistent kernel and its merge kernel, or the cluster kernel, as the call is routed); CUDA events on their stream"}
     if isolated is not None:
         roof["isolated_call_us"] = isolated
     clocks = dict(sampler.summary(), window="1 s of identical steps before and through the timed region"
